@@ -1,0 +1,230 @@
+// fp64 CPU oracle for the bidirectional multi-head self-attention core of a
+// ViT / SigLIP vision encoder.  TEST INFRASTRUCTURE ONLY: the tests, the smoke
+// check and the benchmark's CPU-baseline leg call it; the CUDA library never
+// does, and it shares no code, header or constant with the CUDA path.
+//
+// What it computes (the plain definition, written out with no tiling, no
+// fusion and no reordering):
+//
+//   for every image b, head h and query token i:
+//     s_j  = scale * sum_c q[b,i,h,c] * k[b,j,h,c]          j = 0..N-1
+//     m    = max_j s_j
+//     p_j  = exp(s_j - m)
+//     l    = sum_j p_j
+//     o[b,i,h,c] = (sum_j p_j * v[b,j,h,c]) / l
+//
+// Sources:
+//  * "Pi0 VLA deployment tutorial: Flash Attention for the vision encoder",
+//    section 1: the encoder's time goes to the multi-head self-attention
+//    layers of the ViT backbone, and Flash Attention changes only the memory
+//    access pattern, not the output quality -- so the fused kernel must reach
+//    this same result up to rounding.
+//  * Same page, section 3.2: the ViT block's qkv linear feeds the attention
+//    module (nn.MultiheadAttention swapped for FlashMHA); every patch token and
+//    the CLS token attend to every token (bidirectional, no mask), dropout is
+//    the inference value 0.
+//  * "Pi0 VLA latency report on a 16 GB GPU", section 3.1: ViT-L/14 vision
+//    tower over three 224x224 camera views.
+//  The pages never print the formula; the scaled dot-product softmax above is
+//  the computation nn.MultiheadAttention / FlashMHA perform.
+//
+// Inputs arrive either as fp64 arrays or as the packed [B,N,3,H,d] bf16 bit
+// patterns that the qkv linear emits; bf16 is widened to fp64 exactly.
+// Everything is accumulated and returned in fp64.  Work is spread over
+// (b, h) pairs with std::thread; each (b, h) is computed by one thread in the
+// order written above.
+
+#include <algorithm>
+#include <atomic>
+#include <cmath>
+#include <cstddef>
+#include <cstdint>
+#include <cstring>
+#include <thread>
+#include <vector>
+
+namespace {
+
+double widen_bf16(uint16_t bits) {
+  uint32_t u = static_cast<uint32_t>(bits) << 16;
+  float f;
+  std::memcpy(&f, &u, sizeof(f));
+  return static_cast<double>(f);
+}
+
+// One query row of one head.  qi points at the query's d channels; k and v
+// point at key/value token 0, consecutive tokens `tok_stride` doubles apart,
+// channels contiguous.  Writes d outputs to `oi`; if `probs` is non-null it
+// also receives the N softmax weights of this row.  `s` is N doubles of
+// workspace.
+void one_row(const double* qi, const double* k, const double* v,
+             std::ptrdiff_t tok_stride, int N, int d, double scale,
+             double* oi, double* probs, double* s) {
+  for (int j = 0; j < N; ++j) {
+    const double* kj = k + j * tok_stride;
+    double dot = 0.0;
+    for (int c = 0; c < d; ++c) dot += qi[c] * kj[c];
+    s[j] = scale * dot;
+  }
+  double m = s[0];
+  for (int j = 1; j < N; ++j) m = std::max(m, s[j]);
+  double l = 0.0;
+  for (int j = 0; j < N; ++j) {
+    s[j] = std::exp(s[j] - m);
+    l += s[j];
+  }
+  for (int c = 0; c < d; ++c) {
+    double acc = 0.0;
+    for (int j = 0; j < N; ++j) acc += s[j] * v[j * tok_stride + c];
+    oi[c] = acc / l;
+  }
+  if (probs != nullptr) {
+    for (int j = 0; j < N; ++j) probs[j] = s[j] / l;
+  }
+}
+
+// One (b, h) head: all N query rows.  Outputs have token stride `o_stride`;
+// `probs`, if non-null, receives the N x N softmax matrix (row i = query i).
+void one_head(const double* q, const double* k, const double* v,
+              std::ptrdiff_t tok_stride, int N, int d, double scale,
+              double* o, std::ptrdiff_t o_stride, double* probs) {
+  std::vector<double> s(static_cast<size_t>(N));
+  for (int i = 0; i < N; ++i) {
+    one_row(q + i * tok_stride, k, v, tok_stride, N, d, scale, o + i * o_stride,
+            probs ? probs + static_cast<size_t>(i) * N : nullptr, s.data());
+  }
+}
+
+template <class F>
+void parallel_for(long count, int nthreads, F&& body) {
+  if (nthreads <= 0) {
+    unsigned hc = std::thread::hardware_concurrency();
+    nthreads = hc == 0 ? 1 : static_cast<int>(hc);
+  }
+  nthreads = static_cast<int>(std::min<long>(nthreads, std::max<long>(count, 1)));
+  if (nthreads <= 1) {
+    for (long t = 0; t < count; ++t) body(t);
+    return;
+  }
+  std::atomic<long> next{0};
+  std::vector<std::thread> pool;
+  pool.reserve(static_cast<size_t>(nthreads));
+  for (int w = 0; w < nthreads; ++w) {
+    pool.emplace_back([&]() {
+      for (long t = next.fetch_add(1); t < count; t = next.fetch_add(1)) body(t);
+    });
+  }
+  for (auto& th : pool) th.join();
+}
+
+bool bad_shape(int B, int N, int H, int d) {
+  return B < 0 || N < 0 || H < 0 || d <= 0;
+}
+
+}  // namespace
+
+extern "C" {
+
+// Number of worker threads a call with nthreads <= 0 uses.
+int oracle_default_threads(void) {
+  unsigned hc = std::thread::hardware_concurrency();
+  return hc == 0 ? 1 : static_cast<int>(hc);
+}
+
+// q, k, v, o: contiguous fp64 [B, N, H, d].  Returns 0, or -1 on bad input.
+int oracle_attn_f64(const double* q, const double* k, const double* v, double* o,
+                    int B, int N, int H, int d, double scale, int nthreads) {
+  if (bad_shape(B, N, H, d)) return -1;
+  if (static_cast<long>(B) * N * H == 0) return 0;
+  if (!q || !k || !v || !o) return -1;
+  const std::ptrdiff_t tok = static_cast<std::ptrdiff_t>(H) * d;
+  parallel_for(static_cast<long>(B) * H, nthreads, [&](long t) {
+    const long b = t / H, h = t % H;
+    const std::ptrdiff_t base = b * static_cast<std::ptrdiff_t>(N) * tok + h * d;
+    one_head(q + base, k + base, v + base, tok, N, d, scale, o + base, tok, nullptr);
+  });
+  return 0;
+}
+
+// Softmax matrix: q, k contiguous fp64 [B, N, H, d]; p receives [B, H, N, N].
+int oracle_attn_probs_f64(const double* q, const double* k, double* p,
+                          int B, int N, int H, int d, double scale) {
+  if (bad_shape(B, N, H, d)) return -1;
+  if (static_cast<long>(B) * N * H == 0) return 0;
+  if (!q || !k || !p) return -1;
+  const std::ptrdiff_t tok = static_cast<std::ptrdiff_t>(H) * d;
+  std::vector<double> scratch(static_cast<size_t>(N) * d);
+  for (long b = 0; b < B; ++b) {
+    for (long h = 0; h < H; ++h) {
+      const std::ptrdiff_t base = b * static_cast<std::ptrdiff_t>(N) * tok + h * d;
+      // v is irrelevant for the probabilities; reuse k as a stand-in.
+      one_head(q + base, k + base, k + base, tok, N, d, scale, scratch.data(), d,
+               p + (b * H + h) * static_cast<std::ptrdiff_t>(N) * N);
+    }
+  }
+  return 0;
+}
+
+namespace {
+
+// Widen the (b, h) slice of a packed [B,N,3,H,d] bf16 buffer into three
+// contiguous N x d fp64 arrays.
+void widen_head(const uint16_t* qkv, long b, long h, int N, int H, int d,
+                std::vector<double>& q, std::vector<double>& k, std::vector<double>& v) {
+  const std::ptrdiff_t tok = 3 * static_cast<std::ptrdiff_t>(H) * d;
+  const std::ptrdiff_t hd = static_cast<std::ptrdiff_t>(H) * d;
+  for (int n = 0; n < N; ++n) {
+    const uint16_t* row = qkv + (b * N + n) * tok + h * d;
+    for (int c = 0; c < d; ++c) {
+      q[static_cast<size_t>(n) * d + c] = widen_bf16(row[c]);
+      k[static_cast<size_t>(n) * d + c] = widen_bf16(row[hd + c]);
+      v[static_cast<size_t>(n) * d + c] = widen_bf16(row[2 * hd + c]);
+    }
+  }
+}
+
+}  // namespace
+
+// qkv: packed [B, N, 3, H, d] bf16 bit patterns; o: fp64 [B, N, H, d].
+int oracle_attn_packed_bf16(const uint16_t* qkv, double* o, int B, int N, int H, int d,
+                            double scale, int nthreads) {
+  if (bad_shape(B, N, H, d)) return -1;
+  if (static_cast<long>(B) * N * H == 0) return 0;
+  if (!qkv || !o) return -1;
+  const std::ptrdiff_t otok = static_cast<std::ptrdiff_t>(H) * d;
+  parallel_for(static_cast<long>(B) * H, nthreads, [&](long t) {
+    const long b = t / H, h = t % H;
+    std::vector<double> q(static_cast<size_t>(N) * d), k(q.size()), v(q.size());
+    widen_head(qkv, b, h, N, H, d, q, k, v);
+    one_head(q.data(), k.data(), v.data(), d, N, d, scale,
+             o + b * static_cast<std::ptrdiff_t>(N) * otok + h * d, otok, nullptr);
+  });
+  return 0;
+}
+
+// Selected output rows of a packed bf16 input: rows[3*r .. 3*r+2] = (b, h, n).
+// out receives nrows x d fp64 values, each computed by the plain definition
+// over the whole (b, h) head.
+int oracle_attn_rows_packed_bf16(const uint16_t* qkv, int B, int N, int H, int d,
+                                 double scale, const int64_t* rows, int nrows,
+                                 double* out, int nthreads) {
+  if (bad_shape(B, N, H, d) || nrows < 0) return -1;
+  if (nrows == 0) return 0;
+  if (!qkv || !rows || !out) return -1;
+  for (int r = 0; r < nrows; ++r) {
+    if (rows[3 * r] < 0 || rows[3 * r] >= B || rows[3 * r + 1] < 0 || rows[3 * r + 1] >= H ||
+        rows[3 * r + 2] < 0 || rows[3 * r + 2] >= N)
+      return -1;
+  }
+  parallel_for(nrows, nthreads, [&](long r) {
+    const long b = rows[3 * r], h = rows[3 * r + 1], n = rows[3 * r + 2];
+    std::vector<double> q(static_cast<size_t>(N) * d), k(q.size()), v(q.size());
+    std::vector<double> s(static_cast<size_t>(N));
+    widen_head(qkv, b, h, N, H, d, q, k, v);
+    one_row(q.data() + n * d, k.data(), v.data(), d, N, d, scale, out + r * d, nullptr,
+            s.data());
+  });
+  return 0;
+}
+
+}  // extern "C"

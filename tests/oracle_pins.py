@@ -1,0 +1,265 @@
+"""Checks that pin the fp64 oracle to facts fixed outside itself.
+
+Each ``pin_*`` function takes an ``oracle.OracleLib`` and raises
+``AssertionError`` when the library disagrees with a closed form, a worked
+example, an invariant of the attention definition, a pure-Python brute force
+or PyTorch's own CPU scaled-dot-product attention.  ``test_oracle_pins`` runs
+them against the real oracle; ``test_oracle_mutants`` runs them against
+deliberately broken copies of the oracle source and requires each copy to fail
+at least one pin.
+
+Definition being pinned (multi-head self-attention of the ViT block, as in the
+Pi0 Flash Attention tutorial, sections 1 and 3.2):
+``o[b,i,h,:] = sum_j softmax_j(scale * q[b,i,h,:] . k[b,j,h,:]) v[b,j,h,:]``.
+"""
+from __future__ import annotations
+
+import json
+import math
+import os
+
+import numpy as np
+
+import seeded_inputs as si
+
+GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden", "closed_forms.json")
+
+
+def _rng(seed: int) -> np.random.Generator:
+    return np.random.default_rng(seed)
+
+
+def _close(a, b, tol, what):
+    a = np.asarray(a, dtype=np.float64)
+    b = np.asarray(b, dtype=np.float64)
+    assert a.shape == b.shape, f"{what}: shape {a.shape} != {b.shape}"
+    assert np.all(np.isfinite(a)), f"{what}: non-finite values"
+    err = float(np.max(np.abs(a - b))) if a.size else 0.0
+    assert err <= tol, f"{what}: max |err| {err:.3e} > {tol:.1e}"
+
+
+def pin_golden_closed_forms(lib):
+    """Hand-derived worked examples (tests/golden/closed_forms.json)."""
+    with open(GOLDEN) as f:
+        cases = json.load(f)["cases"]
+    for c in cases:
+        k = np.array(c["k"], dtype=np.float64)
+        v = np.array(c["v"], dtype=np.float64)
+        q = np.array(c["q"], dtype=np.float64)
+        if q.shape[0] < k.shape[0]:
+            q = np.repeat(q, k.shape[0], axis=0)[: k.shape[0]]
+        want = np.array(c["o"], dtype=np.float64)
+        if want.shape[0] < k.shape[0]:
+            want = np.repeat(want, k.shape[0], axis=0)[: k.shape[0]]
+        o = lib.attention_f64(q[None, :, None, :], k[None, :, None, :], v[None, :, None, :],
+                              c["scale"])
+        _close(o[0, :, 0, :], want, c["tol"], c["name"])
+
+
+def pin_single_token(lib):
+    """N = 1: the only weight is 1, so o equals the value row exactly."""
+    r = _rng(1)
+    q, k, v = (r.standard_normal((3, 1, 4, 72)) for _ in range(3))
+    o = lib.attention_f64(q, k, v, 0.3)
+    _close(o, v, 0.0, "N=1 -> o == v")
+
+
+def pin_two_tokens_sigmoid(lib):
+    """N = 2: o_i = sigmoid(s_i0 - s_i1) v_0 + sigmoid(s_i1 - s_i0) v_1."""
+    r = _rng(2)
+    q, k, v = (r.standard_normal((2, 2, 3, 8)) for _ in range(3))
+    scale = 0.7
+    o = lib.attention_f64(q, k, v, scale)
+    want = np.empty_like(o)
+    for b in range(2):
+        for h in range(3):
+            for i in range(2):
+                s0 = scale * float(np.dot(q[b, i, h], k[b, 0, h]))
+                s1 = scale * float(np.dot(q[b, i, h], k[b, 1, h]))
+                w0 = 1.0 / (1.0 + math.exp(s1 - s0))
+                w1 = 1.0 / (1.0 + math.exp(s0 - s1))
+                want[b, i, h] = w0 * v[b, 0, h] + w1 * v[b, 1, h]
+    _close(o, want, 1e-14, "N=2 sigmoid closed form")
+
+
+def pin_identical_values(lib):
+    """Every value row equal to one vector u: the weights sum to 1, so o rows equal u."""
+    r = _rng(3)
+    B, N, H, d = 2, 37, 3, 16
+    q, k = r.standard_normal((B, N, H, d)), r.standard_normal((B, N, H, d))
+    u = r.standard_normal((B, 1, H, d))
+    v = np.broadcast_to(u, (B, N, H, d)).copy()
+    o = lib.attention_f64(q, k, v, 1.3)
+    _close(o, v, 1e-13, "identical V rows")
+
+
+def pin_zero_query_mean(lib):
+    """Q = 0: all logits are 0, so o is the plain mean of the value rows."""
+    r = _rng(4)
+    B, N, H, d = 2, 29, 2, 8
+    q = np.zeros((B, N, H, d))
+    k, v = r.standard_normal((B, N, H, d)), r.standard_normal((B, N, H, d))
+    o = lib.attention_f64(q, k, v, 0.125)
+    want = np.broadcast_to(v.mean(axis=1, keepdims=True), v.shape)
+    _close(o, want, 1e-14, "Q=0 -> mean of V")
+
+
+def pin_probs_rows(lib):
+    """Softmax rows are non-negative, sum to 1, and are proportional to exp(logit)."""
+    r = _rng(5)
+    B, N, H, d = 2, 19, 2, 8
+    q, k = r.standard_normal((B, N, H, d)), r.standard_normal((B, N, H, d))
+    scale = 0.9
+    p = lib.probs_f64(q, k, scale)
+    assert np.all(p >= 0.0), "negative softmax weight"
+    _close(p.sum(axis=-1), np.ones((B, H, N)), 1e-14, "softmax rows sum to 1")
+    s = scale * np.einsum("bihc,bjhc->bhij", q, k)
+    # log-ratio test: log p_ij - log p_i0 == s_ij - s_i0
+    _close(np.log(p) - np.log(p[..., :1]), s - s[..., :1], 1e-12, "softmax log-ratios")
+
+
+def pin_joint_kv_permutation(lib):
+    """Permuting the key and value rows by the same permutation leaves o unchanged;
+    permuting the query rows permutes the output rows."""
+    r = _rng(6)
+    B, N, H, d = 2, 23, 2, 8
+    q, k, v = (r.standard_normal((B, N, H, d)) for _ in range(3))
+    o = lib.attention_f64(q, k, v, 0.5)
+    perm = r.permutation(N)
+    o2 = lib.attention_f64(q, k[:, perm], v[:, perm], 0.5)
+    _close(o2, o, 1e-13, "joint K/V permutation")
+    o3 = lib.attention_f64(q[:, perm], k, v, 0.5)
+    _close(o3, o[:, perm], 1e-13, "query permutation equivariance")
+    # permuting only V must change the result (a K/V mix-up would hide here)
+    o4 = lib.attention_f64(q, k, v[:, perm], 0.5)
+    assert np.max(np.abs(o4 - o)) > 1e-3, "o does not depend on which value row goes with which key"
+
+
+def pin_head_batch_independence(lib):
+    """Each (b, h) slice is computed on its own: it equals a B = H = 1 call on that slice."""
+    r = _rng(7)
+    B, N, H, d = 3, 21, 4, 8
+    q, k, v = (r.standard_normal((B, N, H, d)) for _ in range(3))
+    o = lib.attention_f64(q, k, v, 0.6)
+    for b in range(B):
+        for h in range(H):
+            sl = (slice(b, b + 1), slice(None), slice(h, h + 1), slice(None))
+            oh = lib.attention_f64(q[sl], k[sl], v[sl], 0.6)
+            _close(oh, o[sl], 0.0, f"slice b={b} h={h}")
+
+
+def pin_hard_attention(lib):
+    """A large scale with a unique maximising key gives that key's value row."""
+    r = _rng(8)
+    B, N, H, d = 1, 40, 2, 8
+    q, k, v = (r.standard_normal((B, N, H, d)) for _ in range(3))
+    scale = 1.0e4
+    o = lib.attention_f64(q, k, v, scale)
+    s = np.einsum("bihc,bjhc->bhij", q, k)
+    top = np.argsort(s, axis=-1)
+    for b in range(B):
+        for h in range(H):
+            for i in range(N):
+                j1, j2 = top[b, h, i, -1], top[b, h, i, -2]
+                gap = scale * (s[b, h, i, j1] - s[b, h, i, j2])
+                if gap > 60.0:  # every other weight below e^-60
+                    _close(o[b, i, h], v[b, j1, h], 1e-15, f"hard attention row {i}")
+
+
+def pin_brute_force_python(lib):
+    """Pure-Python loops over a tiny problem, written from the definition."""
+    r = _rng(9)
+    B, N, H, d = 2, 5, 2, 3
+    q, k, v = (r.standard_normal((B, N, H, d)) for _ in range(3))
+    scale = 0.8
+    o = lib.attention_f64(q, k, v, scale)
+    want = np.zeros_like(o)
+    for b in range(B):
+        for h in range(H):
+            for i in range(N):
+                logits = [scale * sum(q[b, i, h, c] * k[b, j, h, c] for c in range(d))
+                          for j in range(N)]
+                w = [math.exp(x) for x in logits]
+                tot = math.fsum(w)
+                for c in range(d):
+                    want[b, i, h, c] = math.fsum(w[j] * v[b, j, h, c] for j in range(N)) / tot
+    _close(o, want, 1e-14, "pure-Python brute force")
+
+
+def _torch_sdpa(q, k, v, scale):
+    import torch
+    import torch.nn.functional as F
+    t = lambda a: torch.from_numpy(np.ascontiguousarray(a)).permute(0, 2, 1, 3)  # [B,H,N,d]
+    o = F.scaled_dot_product_attention(t(q), t(k), t(v), scale=scale)
+    return o.permute(0, 2, 1, 3).contiguous().numpy()
+
+
+def _widen(bits):
+    return si.bf16_bits_to_f32(bits).astype(np.float64)
+
+
+def pin_torch_sdpa_configs(lib, configs=(1, 2, 3, 4)):
+    """PyTorch's CPU scaled_dot_product_attention in fp64 on the seeded config inputs,
+    sliced from the packed buffer by numpy (independently of the oracle's own slicing)."""
+    for ci in configs:
+        c = si.CONFIGS[ci - 1]
+        bits = c.qkv(0)
+        x = _widen(bits)
+        q, k, v = x[:, :, 0], x[:, :, 1], x[:, :, 2]
+        want = _torch_sdpa(q, k, v, c.scale)
+        got = lib.attention_packed_bf16(bits, c.scale)
+        _close(got, want, 1e-12, f"config {ci} vs torch SDPA fp64")
+        got2 = lib.attention_f64(q, k, v, c.scale)
+        _close(got2, want, 1e-12, f"config {ci} fp64 entry vs torch SDPA fp64")
+
+
+def pin_torch_sdpa_large_slice(lib):
+    """One image of the 336px ViT-L/14 shape (N = 577, H = 16, d = 64) against torch SDPA."""
+    c = si.CONFIGS[4]
+    bits = si.packed_qkv(1, c.N, c.H, c.d, c.seed(0))
+    x = _widen(bits)
+    want = _torch_sdpa(x[:, :, 0], x[:, :, 1], x[:, :, 2], c.scale)
+    got = lib.attention_packed_bf16(bits, c.scale)
+    _close(got, want, 1e-12, "N=577 slice vs torch SDPA fp64")
+
+
+def pin_d72_zero_padding(lib):
+    """Zero channels appended to q, k and v (72 -> 80) change neither the logits nor the
+    first 72 output channels, provided the scale stays 1/sqrt(72)."""
+    r = _rng(10)
+    B, N, H = 2, 33, 2
+    q, k, v = (r.standard_normal((B, N, H, 72)) for _ in range(3))
+    scale = 1.0 / math.sqrt(72.0)
+    o = lib.attention_f64(q, k, v, scale)
+    pad = lambda a: np.concatenate([a, np.zeros((B, N, H, 8))], axis=-1)
+    o80 = lib.attention_f64(pad(q), pad(k), pad(v), scale)
+    _close(o80[..., :72], o, 1e-15, "72 -> 80 zero padding")
+    _close(o80[..., 72:], np.zeros((B, N, H, 8)), 0.0, "padded channels stay zero")
+
+
+def pin_rows_entry(lib):
+    """The sampled-rows entry returns exactly the full computation's rows."""
+    c = si.CONFIGS[2]
+    bits = c.qkv(3)
+    full = lib.attention_packed_bf16(bits, c.scale)
+    rows = [(0, 0, 0), (2, 15, 256), (1, 7, 128), (2, 3, 1)]
+    got = lib.attention_rows_packed_bf16(bits, c.scale, rows)
+    for r_, (b, h, n) in enumerate(rows):
+        _close(got[r_], full[b, n, h], 0.0, f"row {(b, h, n)}")
+
+
+ALL_PINS = [
+    pin_golden_closed_forms,
+    pin_single_token,
+    pin_two_tokens_sigmoid,
+    pin_identical_values,
+    pin_zero_query_mean,
+    pin_probs_rows,
+    pin_joint_kv_permutation,
+    pin_head_batch_independence,
+    pin_hard_attention,
+    pin_brute_force_python,
+    pin_torch_sdpa_configs,
+    pin_d72_zero_padding,
+    pin_rows_entry,
+]

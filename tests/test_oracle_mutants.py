@@ -1,0 +1,65 @@
+"""Plant plausible mistakes in copies of the oracle source and show the pins catch each.
+
+Every mutant is compiled from a copy of ``oracle/vla_attn_oracle.cpp`` in a
+temporary directory (the real oracle is never touched) and run through the pin
+suite; the test passes only if at least one pin fails for every mutant.
+"""
+import os
+import shutil
+import subprocess
+
+import pytest
+
+import oracle
+from oracle import build as oracle_build
+from oracle_pins import ALL_PINS
+
+# (name, original text, replacement) -- each a mistake someone could plausibly make.
+MUTANTS = [
+    ("scale_dropped", "s[j] = scale * dot;", "s[j] = dot;"),
+    ("scale_squared", "s[j] = scale * dot;", "s[j] = scale * scale * dot;"),
+    ("key_index_is_query_index", "const double* kj = k + j * tok_stride;",
+     "const double* kj = k + (j == 0 ? 0 : j - 1) * tok_stride;"),
+    ("no_normalisation", "oi[c] = acc / l;", "oi[c] = acc;"),
+    ("value_channels_reversed", "acc += s[j] * v[j * tok_stride + c];",
+     "acc += s[j] * v[j * tok_stride + (d - 1 - c)];"),
+    ("last_key_dropped_from_softmax", "for (int j = 0; j < N; ++j) {\n    s[j] = std::exp(s[j] - m);",
+     "for (int j = 0; j < N - 1; ++j) {\n    s[j] = std::exp(s[j] - m);"),
+    ("no_max_subtraction", "s[j] = std::exp(s[j] - m);", "s[j] = std::exp(s[j]);"),
+    ("sign_flip_logits", "s[j] = scale * dot;", "s[j] = -scale * dot;"),
+    ("k_and_v_slots_swapped", "k[static_cast<size_t>(n) * d + c] = widen_bf16(row[hd + c]);",
+     "k[static_cast<size_t>(n) * d + c] = widen_bf16(row[2 * hd + c]);"),
+    ("head_offset_ignored", "const uint16_t* row = qkv + (b * N + n) * tok + h * d;",
+     "const uint16_t* row = qkv + (b * N + n) * tok;"),
+    ("weights_not_exponentiated_in_probs", "for (int j = 0; j < N; ++j) probs[j] = s[j] / l;",
+     "for (int j = 0; j < N; ++j) probs[j] = s[j];"),
+]
+
+
+@pytest.fixture(scope="module")
+def source():
+    with open(oracle.SOURCE) as f:
+        return f.read()
+
+
+@pytest.mark.parametrize("name,old,new", MUTANTS, ids=[m[0] for m in MUTANTS])
+def test_mutant_is_caught(tmp_path, source, name, old, new):
+    if shutil.which("g++") is None:
+        pytest.skip("g++ not available")
+    assert old in source, f"mutation site for {name} no longer in the oracle source"
+    src = tmp_path / f"mutant_{name}.cpp"
+    src.write_text(source.replace(old, new, 1))
+    lib_path = str(tmp_path / f"libmutant_{name}.so")
+    try:
+        oracle_build.compile_source(str(src), lib_path)
+    except subprocess.CalledProcessError:
+        pytest.fail(f"mutant {name} does not compile")
+    lib = oracle.OracleLib(lib_path)
+    failed = []
+    for pin in ALL_PINS:
+        try:
+            pin(lib)
+        except (AssertionError, ValueError, FloatingPointError):
+            failed.append(pin.__name__)
+    assert failed, f"no pin caught mutant {name}"
+    os.remove(lib_path)
