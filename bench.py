@@ -1,0 +1,363 @@
+"""Benchmark of the B200 attention core on the 336 px ViT-L/14 batch.
+
+Workload: B=256 images, N=577 tokens (576 patches + CLS), H=16 heads, d=64,
+packed bf16 QKV drawn by the seeded generator (synthetic data of the encoder's
+shape).  One step = one call of the fused attention kernel over the whole
+batch.  Prints ONE JSON line (rank 0).
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Under torchrun every rank runs the same per-GPU batch on its own GPU (weak
+scaling, no collective on the data path); the elapsed time is the max over
+ranks.  ``--impl reference`` times the fp64 CPU oracle on the host cores on a
+bounded sample of the same workload (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import glob
+import hashlib
+import json
+import os
+import re
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import seeded_inputs as si  # noqa: E402
+
+WORKLOAD = si.CONFIGS[4]  # vit_l14_336px_b256
+METRIC = "attention TFLOP/s (4*B*H*N^2*d per call) on B200"
+UNIT = "TFLOP/s"
+KERNEL_SOURCES = ["vit_self_attention_b200/csrc/attn_kernel.cuh",
+                  "vit_self_attention_b200/csrc/ptx.cuh",
+                  "vit_self_attention_b200/csrc/vla_attn.cu"]
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    for rel in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def measured_peaks() -> dict:
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return {"bf16_tflops": float(d["bf16_tflops"]),
+                "bf16_tflops_sustained": float(d.get("bf16_tflops_sustained", d["bf16_tflops"])),
+                "hbm_gbs": float(d["hbm_gbs"]), "source": "measured"}
+    return {"bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "hbm_gbs": 6650.0,
+            "source": "fallback"}
+
+
+def ncu_traffic(workload: str) -> tuple[float | None, str | None]:
+    """DRAM bytes per launch from the committed ncu summary of this kernel and workload,
+    if it was taken on the current kernel source (else None)."""
+    cur = kernel_source_hash()
+    for path in sorted(glob.glob(os.path.join(ROOT, "profiles", "*.md"))):
+        with open(path) as f:
+            txt = f.read()
+        m_w = re.search(r"^workload:\s*(\S+)", txt, re.M)
+        m_h = re.search(r"^kernel_source_sha256_16:\s*([0-9a-f]+)", txt, re.M)
+        m_t = re.search(r"^dram_bytes_per_full_launch:\s*([0-9.eE+]+)", txt, re.M)
+        if m_w and m_h and m_t and m_w.group(1) == workload and m_h.group(1) == cur:
+            return float(m_t.group(1)), os.path.relpath(path, ROOT)
+    return None, None
+
+
+_REASON_BITS = {
+    0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+    0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+    0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting",
+}
+
+
+class ClockSampler:
+    """Samples SM clock and throttle reasons through NVML while the timed region runs."""
+
+    def __init__(self, device_index: int, period_s: float = 0.005):
+        self.samples: list[tuple[int, int]] = []
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._period = period_s
+        self._ok = False
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self._nvml = pynvml
+            self._h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = int(pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM))
+            self._ok = True
+        except Exception:  # NVML missing: report no clocks
+            self._ok = False
+        self._t = threading.Thread(target=self._run, daemon=True)
+
+    def _run(self):
+        nv = self._nvml
+        while not self._stop.is_set():
+            try:
+                mhz = int(nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM))
+                reasons = int(nv.nvmlDeviceGetCurrentClocksEventReasons(self._h))
+                self.samples.append((mhz, reasons))
+            except Exception:
+                pass
+            time.sleep(self._period)
+
+    def __enter__(self):
+        if self._ok:
+            self._t.start()
+        return self
+
+    def __exit__(self, *exc):
+        self._stop.set()
+        if self._ok:
+            self._t.join()
+
+    def summary(self) -> dict | None:
+        if not self._ok or not self.samples:
+            return None
+        mhz = [m for m, _ in self.samples]
+        seen = 0
+        for _, r in self.samples:
+            seen |= r
+        names = sorted(n for bit, n in _REASON_BITS.items() if seen & bit and n != "gpu_idle")
+        return {"sm_mhz": float(statistics.median(mhz)), "sm_max_mhz": self.max_mhz,
+                "reasons": names, "samples": len(mhz), "sm_mhz_min": min(mhz),
+                "sm_mhz_max_seen": max(mhz)}
+
+
+# ---------------------------------------------------------------- oracle (CPU)
+def cpu_oracle_rate(target_s: float, max_heads: int | None = None) -> dict:
+    """Time the fp64 oracle on whole (b, h) heads of the workload, doubling the sample
+    until one run takes at least target_s; returns TFLOP/s of the last run."""
+    import oracle
+    c = WORKLOAD
+    threads = oracle.default_threads()
+    images = 1
+    bits_cache = {}
+    last = None
+    while True:
+        if images not in bits_cache:
+            bits_cache.clear()
+            bits_cache[images] = si.packed_qkv(images, c.N, c.H, c.d, c.seed(0))
+        bits = bits_cache[images]
+        t0 = time.perf_counter()
+        oracle.attention_packed_bf16(bits, c.scale, threads=threads)
+        dt = time.perf_counter() - t0
+        flops = 4.0 * images * c.H * c.N * c.N * c.d
+        last = {"value": flops / dt / 1e12, "unit": UNIT, "cores": threads, "kind": "oracle",
+                "sample": f"{images} image(s) x {c.H} heads of the B=256 N=577 H=16 d=64 batch "
+                          f"({images * c.H} of {c.B * c.H} heads), fp64, {dt:.2f} s",
+                "seconds": dt}
+        if dt >= target_s or images >= c.B or (max_heads and images * c.H >= max_heads):
+            return last
+        images = min(c.B, images * 2 if dt < target_s / 4 else images + max(1, images // 2))
+
+
+def run_reference(args, rank: int, world: int) -> None:
+    if rank != 0:
+        return
+    c = WORKLOAD
+    import oracle
+    threads = oracle.default_threads()
+    # Size one step so warm-up + timed steps end within about two minutes.
+    per_step = max(0.5, min(5.0, 120.0 / max(1, args.steps + args.warmup)))
+    probe = cpu_oracle_rate(0.2)
+    heads_per_s = probe["value"] * 1e12 / (4.0 * c.N * c.N * c.d)
+    images = int(max(1, min(c.B, round(per_step * heads_per_s / c.H))))
+    bits = si.packed_qkv(images, c.N, c.H, c.d, c.seed(0))
+    for _ in range(args.warmup):
+        oracle.attention_packed_bf16(bits, c.scale, threads=threads)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        oracle.attention_packed_bf16(bits, c.scale, threads=threads)
+    dt = time.perf_counter() - t0
+    flops = 4.0 * images * c.H * c.N * c.N * c.d * args.steps
+    value = flops / dt / 1e12
+    sample = (f"each step: {images} image(s) x {c.H} heads of the B=256 N=577 H=16 d=64 batch, "
+              f"fp64 oracle on {threads} host threads")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded splitmix64 Box-Muller, bf16)",
+        "config": {"workload": c.name, "B": c.B, "N": c.N, "H": c.H, "d": c.d,
+                   "images_per_step": images},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "images_per_s_24_layers": value * 1e12 / (4.0 * c.H * c.N * c.N * c.d) / 24.0,
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------- CUDA path
+def run_ours(args, rank: int, world: int, local_rank: int) -> None:
+    import torch
+    import torch.distributed as dist
+
+    import vit_self_attention_b200 as vab
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    c = WORKLOAD
+    stream = torch.cuda.current_stream(dev)
+
+    bits = si.packed_qkv(c.B, c.N, c.H, c.d, c.seed(0) + 7919 * rank)
+    host_in = torch.from_numpy(bits.view(np.int16)).pin_memory()
+    qkv = host_in.to(dev, non_blocking=False).view(torch.bfloat16)
+    out = torch.empty((c.B, c.N, c.H, c.d), dtype=torch.bfloat16, device=dev)
+    base = qkv.data_ptr()
+    step_b = c.H * c.d * 2
+
+    def step():
+        vab.vla_attn_fwd(base, base + step_b, base + 2 * step_b, out, c.B, c.N, c.H, c.d,
+                         c.scale, stream)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    torch.cuda.synchronize()
+
+    launches0 = vab.vla_attn_launch_count()
+    ev0 = torch.cuda.Event(enable_timing=True)
+    ev1 = torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local_rank) as clocks:
+        barrier()
+        torch.cuda.synchronize()
+        ev0.record(stream)
+        for _ in range(args.steps):
+            step()
+        ev1.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+    launches = vab.vla_attn_launch_count() - launches0
+    ms = ev0.elapsed_time(ev1)
+    st, site = vab.vla_attn_last_device_status(stream)
+    if st != 0:
+        raise RuntimeError(f"device status {st} (site {site}) after the timed region")
+
+    # ---- end-to-end through the host-buffer C-ABI entry (pinned host memory)
+    host_out = torch.empty((c.B, c.N, c.H, c.d), dtype=torch.int16).pin_memory()
+    dev_in = torch.empty(bits.shape, dtype=torch.int16, device=dev)
+    dev_out = torch.empty((c.B, c.N, c.H, c.d), dtype=torch.int16, device=dev)
+    e2e_steps = max(2, min(args.steps, 10))
+
+    def e2e_step():
+        vab.vla_attn_fwd_host(host_in, host_out, dev_in, dev_out, c.B, c.N, c.H, c.d, c.scale,
+                              stream)
+
+    e2e_step()
+    torch.cuda.synchronize()
+    barrier()
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    e2e_ms = e0.elapsed_time(e1)
+
+    if world > 1:
+        t = torch.tensor([ms, e2e_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms, e2e_ms = float(t[0]), float(t[1])
+
+    flops_call = float(c.flops())
+    ms_step = ms / args.steps
+    value = flops_call * world * args.steps / (ms / 1e3) / 1e12
+    e2e_value = flops_call * world * e2e_steps / (e2e_ms / 1e3) / 1e12
+    peaks = measured_peaks()
+    achieved = flops_call / (ms_step / 1e3) / 1e12
+    traffic, traffic_src = ncu_traffic(c.name)
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cb = cpu_oracle_rate(args.cpu_seconds)
+        cpu = {k: cb[k] for k in ("value", "unit", "cores", "kind", "sample")}
+    if rank != 0:
+        return
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": max(3, args.warmup), "ms_per_step": ms_step, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded splitmix64 Box-Muller, bf16)",
+        "config": {"workload": c.name, "B": c.B, "N": c.N, "H": c.H, "d": c.d,
+                   "scale": c.scale, "flops_per_call": c.flops(),
+                   "hbm_bytes_per_call": c.bytes(),
+                   "l2": "inputs larger than L2 (1.21 GB of QKV + O per step vs 126 MB L2)"},
+        "images_per_s_24_layers": world * c.B / (ms_step / 1e3) / 24.0,
+        "roofline": {"bound": "tensor", "achieved": achieved,
+                     "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                     "frac": achieved / peaks["bf16_tflops"], "traffic": traffic,
+                     "peak_source": f"{peaks['source']} bf16 burst (cuBLAS)",
+                     "frac_of_sustained": achieved / peaks["bf16_tflops_sustained"],
+                     "hbm_gbs_achieved": c.bytes() / (ms_step / 1e3) / 1e9,
+                     "traffic_source": traffic_src},
+        "cpu_baseline": cpu,
+        "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": int(bits.nbytes),
+                "d2h_bytes_per_step": int(c.B * c.N * c.H * c.d * 2),
+                "steps": e2e_steps, "ms_per_step": e2e_ms / e2e_steps,
+                "api": "vla_attn_fwd_host (pinned host buffers)"},
+        "gpu_launches": int(launches),
+        "clocks": clocks.summary(),
+        "kernel_source_sha256_16": kernel_source_hash(),
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main() -> None:
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--cpu-seconds", type=float, default=10.0,
+                    help="target duration of the CPU oracle baseline sample")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus and world > 1:
+        print(f"warning: WORLD_SIZE={world} but --gpus {args.gpus}", file=sys.stderr)
+
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+        return
+
+    if world > 1:
+        import datetime
+
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+    try:
+        run_ours(args, rank, world, local_rank)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

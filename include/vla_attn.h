@@ -1,0 +1,127 @@
+/*
+ * vla_attn.h -- C ABI of the B200 (sm_100a) self-attention core of a ViT /
+ * SigLIP vision encoder.
+ *
+ * Operation.  For every image b, head h and query token i of a packed QKV
+ * buffer, the library computes
+ *
+ *     o[b,i,h,:] = sum_j softmax_j( scale * q[b,i,h,:] . k[b,j,h,:] ) v[b,j,h,:]
+ *
+ * over all N tokens of the image (bidirectional, no mask, no dropout).  This
+ * is the multi-head self-attention of the ViT backbone that the Pi0 Flash
+ * Attention tutorial accelerates ("Pi0 VLA deployment tutorial: Flash
+ * Attention for the vision encoder", section 1 for the operation and the
+ * claim that the fused kernel keeps the output unchanged, section 3.2 for the
+ * qkv linear feeding nn.MultiheadAttention / FlashMHA at inference, dropout 0).
+ * The same layers are the ViT-L/14 tower of the "Pi0 VLA latency report on a
+ * 16 GB GPU" (section 3.1) and the SigLIP tower of the Realtime-VLA write-up
+ * (section 1.1.2).
+ *
+ * Data layout.
+ *   q, k, v   point into ONE packed bf16 buffer laid out [B, N, 3, H, d]
+ *             (what the encoder's qkv linear emits, viewed per head):
+ *             k == q + H*d elements, v == q + 2*H*d elements, token stride
+ *             3*H*d elements.  Any other relation is rejected.
+ *   o         separate bf16 buffer [B, N, H, d] (= [B, N, H*d], the input of
+ *             the output projection).
+ *   Arithmetic: bf16 inputs, fp32 accumulation of Q K^T and P V on the tensor
+ *   cores, fp32 online softmax, P rounded to bf16 before P V, O rounded to
+ *   bf16 (nearest even) on store.
+ *
+ * Ownership.  The caller owns every buffer.  vla_attn_fwd allocates no memory,
+ * never synchronises the host, and enqueues exactly one kernel on `stream`
+ * (a cudaStream_t; NULL = the legacy default stream).  All pointers are device
+ * pointers of the current device.
+ *
+ * Errors.  Argument errors are returned synchronously before anything is
+ * enqueued.  A launch failure returns VLA_ATTN_ERR_CUDA.  Every wait inside
+ * the kernel is bounded; a wait that runs out records a code in a device-side
+ * status word, which vla_attn_last_device_status() reports.
+ */
+#ifndef VLA_ATTN_H_
+#define VLA_ATTN_H_
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  VLA_ATTN_OK = 0,
+  VLA_ATTN_ERR_NULL = -1,        /* a required pointer is NULL */
+  VLA_ATTN_ERR_SHAPE = -2,       /* B, N or H < 1, or q/k/v not the packed [B,N,3,H,d] relation */
+  VLA_ATTN_ERR_UNSUPPORTED = -3, /* d not 64 or 72, or N above vla_attn_max_tokens(d) */
+  VLA_ATTN_ERR_ALIGN = -4,       /* q or o not 16-byte aligned */
+  VLA_ATTN_ERR_SCALE = -5,       /* scale not finite or not > 0 */
+  VLA_ATTN_ERR_CUDA = -6,        /* a CUDA runtime / driver call failed */
+  VLA_ATTN_ERR_TIMEOUT = -7,     /* a bounded in-kernel wait ran out (device status) */
+  VLA_ATTN_ERR_DEVICE = -8,      /* current device is not sm_100 (B200 class) */
+  VLA_ATTN_ERR_MEMORY = -9       /* a pointer is not device memory of the current device,
+                                    or its allocation is too small for the shape */
+} vla_attn_status;
+
+/*
+ * Attention forward on the packed QKV buffer (see the header comment).
+ *   q, k, v  device pointers into one [B, N, 3, H, d] bf16 buffer (k = q + H*d,
+ *            v = q + 2*H*d elements); q must be 16-byte aligned.
+ *   o        device pointer to [B, N, H, d] bf16 output, 16-byte aligned; must
+ *            not overlap the input.
+ *   B        images (camera views x batch), >= 1.
+ *   N        tokens per image (patches + CLS), 1 <= N <= vla_attn_max_tokens(d).
+ *   H        heads, >= 1.
+ *   d        head dimension, 64 (ViT-B/16, ViT-L/14) or 72 (SigLIP-So400m/14).
+ *   scale    logit scale, usually 1/sqrt(d); finite and > 0.
+ *   stream   cudaStream_t to enqueue on.
+ * Returns VLA_ATTN_OK or a negative vla_attn_status.
+ */
+int vla_attn_fwd(const void* q, const void* k, const void* v, void* o,
+                 int B, int N, int H, int d, float scale, void* stream);
+
+/*
+ * End-to-end variant for callers whose data live in host memory: copies the
+ * packed [B, N, 3, H, d] bf16 input from `qkv_host` into the caller's device
+ * buffer `qkv_dev`, runs vla_attn_fwd on it into `o_dev`, and copies the
+ * [B, N, H, d] bf16 result back to `o_host` -- all enqueued on `stream`, one
+ * cudaMemcpyAsync per direction.  Host buffers should be pinned
+ * (cudaHostAlloc / cudaHostRegister) for the copies to be asynchronous.  The
+ * host result is valid once the stream has been synchronised.  Same argument
+ * rules and status codes as vla_attn_fwd; allocates nothing.
+ */
+int vla_attn_fwd_host(const void* qkv_host, void* o_host, void* qkv_dev, void* o_dev,
+                      int B, int N, int H, int d, float scale, void* stream);
+
+/* Human-readable text for a status code (static storage, never NULL). */
+const char* vla_attn_strerror(int status);
+
+/*
+ * Synchronises `stream` and returns the device-side status of the kernels run
+ * since the last reset: VLA_ATTN_OK, or VLA_ATTN_ERR_TIMEOUT if a bounded wait
+ * ran out (the output of that launch is then undefined).  `site`, if non-NULL,
+ * receives the code of the first wait that ran out (0 if none).
+ */
+int vla_attn_last_device_status(void* stream, int* site);
+
+/* Clears the device-side status word of the current device (enqueued on `stream`). */
+int vla_attn_reset_device_status(void* stream);
+
+/* Largest N the kernels accept for head dimension d (0 if d is unsupported). */
+int vla_attn_max_tokens(int d);
+
+/* Number of kernels this library has launched in this process. */
+uint64_t vla_attn_launch_count(void);
+
+/*
+ * Testing hook: bound (in nanoseconds) of every in-kernel wait for launches
+ * that follow on this host thread's process; 0 restores the default (1 s).
+ * A tiny bound makes waits run out on purpose so that the error path can be
+ * exercised: the kernel then records VLA_ATTN_ERR_TIMEOUT, drains its own
+ * copies and tensor-core work, frees its tensor memory and returns.
+ */
+void vla_attn_set_wait_limit_ns(uint64_t ns);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* VLA_ATTN_H_ */

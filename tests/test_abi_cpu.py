@@ -1,0 +1,118 @@
+"""The C-ABI library loads, exports every declared symbol, and validates arguments
+on the host before touching a GPU (these tests need no GPU)."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "vla_attn.h")
+
+
+def declared_functions():
+    with open(HEADER) as f:
+        text = f.read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(vla_attn_[a-z_]+)\s*\(", text)))
+
+
+def test_header_declares_the_entry_points():
+    names = declared_functions()
+    assert "vla_attn_fwd" in names and "vla_attn_strerror" in names
+    assert len(names) >= 8
+
+
+def test_library_exports_every_declared_symbol():
+    import vit_self_attention_b200 as vab
+    lib = ctypes.CDLL(vab.LIBRARY_PATH)
+    for name in declared_functions():
+        assert hasattr(lib, name), f"{name} not exported"
+    assert set(declared_functions()) == set(vab.EXPORTED_SYMBOLS)
+    nm = subprocess.run(["nm", "-D", "--defined-only", vab.LIBRARY_PATH], capture_output=True,
+                        text=True)
+    if nm.returncode == 0:
+        for name in declared_functions():
+            assert re.search(rf"\bT {name}$", nm.stdout, re.M), f"{name} not a defined text symbol"
+
+
+def test_build_targets_sm100a_only():
+    from vit_self_attention_b200 import build
+    f = build.flags()
+    assert "arch=compute_100a,code=sm_100a" in f
+    assert sum(1 for x in f if x == "-gencode") == 1
+
+
+H, D = 12, 64
+Q = 0x10000000
+K = Q + H * D * 2
+V = Q + 2 * H * D * 2
+O = 0x20000000
+
+
+def call(q=Q, k=K, v=V, o=O, B=1, N=50, h=H, d=D, scale=0.125):
+    import vit_self_attention_b200 as vab
+    return vab.vla_attn_fwd(q, k, v, o, B, N, h, d, scale, stream=0, check=False)
+
+
+def test_argument_validation_on_host():
+    import vit_self_attention_b200 as vab
+    assert call(q=0) == vab.ERR_NULL
+    assert call(o=0) == vab.ERR_NULL
+    assert call(B=0) == vab.ERR_SHAPE
+    assert call(N=0) == vab.ERR_SHAPE
+    assert call(h=0) == vab.ERR_SHAPE
+    assert call(N=-5) == vab.ERR_SHAPE
+    assert call(d=128, k=Q + H * 128 * 2, v=Q + 4 * H * 128) == vab.ERR_UNSUPPORTED
+    assert call(d=32, k=Q + H * 32 * 2, v=Q + 4 * H * 32) == vab.ERR_UNSUPPORTED
+    assert call(N=578) == vab.ERR_UNSUPPORTED
+    assert call(k=K + 2) == vab.ERR_SHAPE          # not the packed relation
+    assert call(v=K) == vab.ERR_SHAPE
+    assert call(q=Q + 2, k=K + 2, v=V + 2) == vab.ERR_ALIGN
+    assert call(o=O + 8) == vab.ERR_ALIGN
+    assert call(scale=0.0) == vab.ERR_SCALE
+    assert call(scale=-1.0) == vab.ERR_SCALE
+    assert call(scale=float("inf")) == vab.ERR_SCALE
+    assert call(scale=float("nan")) == vab.ERR_SCALE
+
+
+def test_valid_arguments_without_gpu_fail_cleanly():
+    import torch
+
+    import vit_self_attention_b200 as vab
+    if torch.cuda.is_available():
+        pytest.skip("this checks the no-GPU path")
+    assert call() in (vab.ERR_CUDA, vab.ERR_DEVICE)
+    assert vab.vla_attn_launch_count() == 0
+
+
+def test_strerror_and_limits():
+    import vit_self_attention_b200 as vab
+    for st in range(-9, 1):
+        assert vab.vla_attn_strerror(st)
+    assert "unknown" in vab.vla_attn_strerror(-99)
+    assert vab.vla_attn_max_tokens(64) == 577 and vab.vla_attn_max_tokens(72) == 577
+    assert vab.vla_attn_max_tokens(128) == 0
+
+
+def test_host_entry_validation():
+    import vit_self_attention_b200 as vab
+    st = vab.vla_attn_fwd_host(0, O, Q, O, 1, 50, H, D, 0.125, stream=0, check=False)
+    assert st == vab.ERR_NULL
+    st = vab.vla_attn_fwd_host(0x1000, 0x2000, Q, O, 1, 50, H, D, -1.0, stream=0, check=False)
+    assert st == vab.ERR_SCALE
+
+
+def test_product_package_has_no_oracle_or_fallback():
+    """The CUDA package never imports the oracle nor carries a CPU/torch compute path."""
+    pkg = os.path.join(ROOT, "vit_self_attention_b200")
+    for dirpath, _, files in os.walk(pkg):
+        for fn in files:
+            if not fn.endswith((".py", ".cu", ".cuh", ".h", ".cpp")):
+                continue
+            with open(os.path.join(dirpath, fn)) as f:
+                src = f.read()
+            assert "oracle" not in src.lower(), f"{fn} mentions the oracle"
+            assert "scaled_dot_product_attention" not in src, f"{fn} has a torch attention path"
+            assert "softmax(" not in src.replace("softmax(Q", "").replace("softmax(q", ""), fn

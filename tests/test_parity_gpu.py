@@ -1,0 +1,201 @@
+"""CUDA path vs. the fp64 oracle on identical seeded inputs (element by element).
+
+Tolerance on the bf16 outputs, per call: max |err| <= 2e-2 and mean |err| <= 2e-3.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import seeded_inputs as si
+from gpu_helpers import assert_parity, device_qkv, needs_gpu, run_cuda
+
+pytestmark = [pytest.mark.gpu, needs_gpu]
+
+
+@pytest.mark.parametrize("cfg", [1, 2, 3, 4])
+def test_configs_every_call(cfg):
+    """Every seeded layer call of the four encoder workloads."""
+    c = si.CONFIGS[cfg - 1]
+    for call in range(c.calls):
+        bits = c.qkv(call)
+        want = oracle.attention_packed_bf16(bits, c.scale)
+        got = run_cuda(bits, c.scale)
+        assert_parity(got, want, f"config {cfg} ({c.name}) call {call}")
+
+
+EDGE_N = [1, 2, 15, 16, 17, 63, 64, 65, 127, 128, 129, 200, 255, 256, 257, 383, 384, 385, 511,
+          512, 513, 576, 577]
+
+
+@pytest.mark.parametrize("d", [64, 72])
+@pytest.mark.parametrize("N", EDGE_N)
+def test_edge_token_counts(N, d):
+    """Ragged query tiles and key blocks, single- and two-slot rounds, ring streaming (d=72, N>512)."""
+    B, H = 2, 3
+    bits = si.packed_qkv(B, N, H, d, seed=70000 + 10 * N + d)
+    scale = 1.0 / math.sqrt(d)
+    want = oracle.attention_packed_bf16(bits, scale)
+    got = run_cuda(bits, scale)
+    assert_parity(got, want, f"B={B} N={N} H={H} d={d}")
+
+
+@pytest.mark.parametrize("B,H,N,d", [(160, 1, 197, 64), (10, 16, 257, 64), (12, 13, 577, 64),
+                                     (75, 2, 577, 72), (1, 1, 577, 64), (148, 1, 129, 72),
+                                     (300, 1, 50, 64)])
+def test_schedules(B, H, N, d):
+    """Whole-head work units (B*H >= #SMs) and per-round units, persistent multi-unit CTAs."""
+    bits = si.packed_qkv(B, N, H, d, seed=90000 + B * 7 + H * 3 + N + d)
+    scale = 1.0 / math.sqrt(d)
+    want = oracle.attention_packed_bf16(bits, scale)
+    got = run_cuda(bits, scale)
+    assert_parity(got, want, f"B={B} N={N} H={H} d={d}")
+
+
+@pytest.mark.parametrize("sigma", [2.0, 4.0])
+@pytest.mark.parametrize("d", [64, 72])
+def test_peaked_softmax(sigma, d):
+    """Large logits: the running maximum grows across key blocks, exercising the O rescale."""
+    B, N, H = 2, 577, 4
+    bits = si.packed_qkv(B, N, H, d, seed=int(50000 + sigma * 10 + d), sigma_qk=sigma)
+    # Make later keys larger so the row maximum keeps growing block after block.
+    x = si.bf16_bits_to_f32(bits).copy()
+    ramp = (1.0 + 2.0 * np.arange(N, dtype=np.float32) / N)[None, :, None, None]
+    x[:, :, 1] *= ramp
+    bits = si.f32_to_bf16_bits(x)
+    scale = 1.0 / math.sqrt(d)
+    want = oracle.attention_packed_bf16(bits, scale)
+    got = run_cuda(bits, scale)
+    assert_parity(got, want, f"sigma={sigma} d={d}")
+
+
+def test_closed_form_inputs_on_gpu():
+    """Identical V rows -> O rows equal V; Q = 0 -> O = mean of V (in bf16 precision)."""
+    B, N, H, d = 2, 300, 2, 64
+    bits = si.packed_qkv(B, N, H, d, seed=4242)
+    x = si.bf16_bits_to_f32(bits).copy()
+    x[:, :, 2] = x[:, :1, 2]  # every value row equals token 0's
+    got = run_cuda(si.f32_to_bf16_bits(x), 0.125)
+    want = np.broadcast_to(x[:, :1, 2], (B, N, H, d)).astype(np.float64)
+    assert_parity(got, want, "identical V rows", max_tol=1e-2, mean_tol=2e-3)
+    x2 = si.bf16_bits_to_f32(bits).copy()
+    x2[:, :, 0] = 0.0
+    got2 = run_cuda(si.f32_to_bf16_bits(x2), 0.125)
+    want2 = np.broadcast_to(x2[:, :, 2].astype(np.float64).mean(axis=1, keepdims=True),
+                            (B, N, H, d))
+    assert_parity(got2, want2, "Q = 0 -> mean of V")
+
+
+def test_large_config_sampled_rows_and_hull():
+    """The 336 px ViT-L/14 batch (B=256, N=577, H=16, d=64) in the bench's launch
+    configuration: complete heads and scattered rows against the oracle, and every
+    output inside the per-channel range of its head's value rows (O is a convex
+    combination of V rows)."""
+    c = si.CONFIGS[4]
+    bits = c.qkv(0)
+    qkv = device_qkv(bits)
+    import vit_self_attention_b200 as vab
+    out = vab.attention(qkv, c.scale)
+    torch.cuda.synchronize()
+    rng = np.random.default_rng(5)
+    rows = [(0, 0, n) for n in range(c.N)] + [(255, 15, n) for n in range(c.N)]
+    for _ in range(512):
+        rows.append((int(rng.integers(0, c.B)), int(rng.integers(0, c.H)), int(rng.integers(0, c.N))))
+    for n in (0, 127, 128, 511, 512, 575, 576):
+        rows.append((int(rng.integers(0, c.B)), int(rng.integers(0, c.H)), n))
+    want = oracle.attention_rows_packed_bf16(bits, c.scale, rows)
+    idx = torch.tensor(rows, dtype=torch.long, device="cuda")
+    got = out[idx[:, 0], idx[:, 2], idx[:, 1]].float().cpu().numpy().astype(np.float64)
+    assert_parity(got, want, "B=256 N=577 sampled rows")
+    v = qkv[:, :, 2].float()  # [B, N, H, d]
+    lo = v.amin(dim=1, keepdim=True)
+    hi = v.amax(dim=1, keepdim=True)
+    of = out.float()
+    assert torch.isfinite(of).all()
+    slack = 1e-2 * (hi - lo) + 1e-3
+    assert bool(((of >= lo - slack) & (of <= hi + slack)).all()), "output outside value hull"
+
+
+def test_graph_capture_replay():
+    """The call can be captured in a CUDA graph and replayed (pointers stay fixed)."""
+    import vit_self_attention_b200 as vab
+    c = si.CONFIGS[2]
+    bits = c.qkv(0)
+    qkv = device_qkv(bits)
+    out = torch.empty((c.B, c.N, c.H, c.d), dtype=torch.bfloat16, device="cuda")
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):
+        vab.attention(qkv, c.scale, out=out, stream=s)  # warm-up outside capture
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s):
+        vab.attention(qkv, c.scale, out=out, stream=s)
+    out.zero_()
+    g.replay()
+    torch.cuda.synchronize()
+    want = oracle.attention_packed_bf16(bits, c.scale)
+    assert_parity(out.float().cpu().numpy().astype(np.float64), want, "graph replay")
+    bits2 = c.qkv(1)
+    qkv.copy_(device_qkv(bits2))
+    g.replay()
+    torch.cuda.synchronize()
+    want2 = oracle.attention_packed_bf16(bits2, c.scale)
+    assert_parity(out.float().cpu().numpy().astype(np.float64), want2, "graph replay, new input")
+
+
+def test_host_buffer_entry():
+    """vla_attn_fwd_host: pinned host input -> device -> kernel -> pinned host output."""
+    import vit_self_attention_b200 as vab
+    c = si.CONFIGS[3]
+    bits = c.qkv(5)
+    host_in = torch.from_numpy(bits.view(np.int16).copy()).pin_memory()
+    host_out = torch.empty((c.B, c.N, c.H, c.d), dtype=torch.int16).pin_memory()
+    dev_in = torch.empty(bits.shape, dtype=torch.int16, device="cuda")
+    dev_out = torch.empty((c.B, c.N, c.H, c.d), dtype=torch.int16, device="cuda")
+    vab.vla_attn_fwd_host(host_in, host_out, dev_in, dev_out, c.B, c.N, c.H, c.d, c.scale)
+    torch.cuda.synchronize()
+    got = si.bf16_bits_to_f32(host_out.numpy().view(np.uint16)).astype(np.float64)
+    want = oracle.attention_packed_bf16(bits, c.scale)
+    assert_parity(got, want, "host-buffer entry")
+
+
+def test_device_status_clean_and_launch_count():
+    import vit_self_attention_b200 as vab
+    n0 = vab.vla_attn_launch_count()
+    run_cuda(si.CONFIGS[0].qkv(0), si.CONFIGS[0].scale)
+    assert vab.vla_attn_launch_count() == n0 + 1
+    st, site = vab.vla_attn_last_device_status()
+    assert st == 0 and site == 0
+
+
+def test_rejects_host_and_short_buffers():
+    """Pointers that are not device memory, allocations too small for the shape, and an
+    output overlapping the input are refused before anything is launched."""
+    import vit_self_attention_b200 as vab
+    from cuda.bindings import runtime as cudart
+    B, N, H, d = 1, 50, 12, 64
+    in_bytes = B * N * 3 * H * d * 2
+    out = torch.empty(B * N * H * d, dtype=torch.bfloat16, device="cuda")
+    err, raw = cudart.cudaMalloc(in_bytes - 256)  # its own allocation, 256 bytes short
+    assert int(err) == 0
+    try:
+        st = vab.vla_attn_fwd(raw, raw + H * d * 2, raw + 2 * H * d * 2, out, B, N, H, d, 0.125,
+                              check=False)
+        assert st == vab.ERR_MEMORY
+    finally:
+        cudart.cudaFree(raw)
+    host = torch.empty(B * N * 3 * H * d, dtype=torch.bfloat16)
+    hb = host.data_ptr()
+    st = vab.vla_attn_fwd(hb, hb + H * d * 2, hb + 2 * H * d * 2, out, B, N, H, d, 0.125,
+                          check=False)
+    assert st == vab.ERR_MEMORY
+    full = torch.empty(B * N * 3 * H * d, dtype=torch.bfloat16, device="cuda")
+    fb = full.data_ptr()
+    st = vab.vla_attn_fwd(fb, fb + H * d * 2, fb + 2 * H * d * 2, fb, B, N, H, d, 0.125,
+                          check=False)
+    assert st == vab.ERR_MEMORY  # output overlapping the input
+    assert vab.vla_attn_fwd(fb, fb + H * d * 2, fb + 2 * H * d * 2, out, B, 578, H, d, 0.125,
+                            check=False) == vab.ERR_UNSUPPORTED
+    assert vab.vla_attn_launch_count() >= 0

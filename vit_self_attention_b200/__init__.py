@@ -1,0 +1,162 @@
+"""B200 (sm_100a) self-attention core of a ViT / SigLIP vision encoder.
+
+Thin ctypes binding over ``libvla_attn.so`` (C ABI in ``include/vla_attn.h``):
+argument marshalling only -- every step of the computation runs in the CUDA
+kernels of that library.  There is no CPU or PyTorch fallback: importing this
+package fails loudly when the library has not been built.
+
+Operation: ``o = softmax(q k^T * scale) v`` per image and head over the packed
+``[B, N, 3, H, d]`` bf16 QKV that a ViT block's qkv linear emits (the
+multi-head self-attention of the Pi0 Flash Attention tutorial, sections 1 and
+3.2), output ``[B, N, H, d]`` bf16.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIBRARY_PATH = os.path.join(_PKG, "libvla_attn.so")
+
+if not os.path.exists(LIBRARY_PATH):
+    raise ImportError(
+        f"{LIBRARY_PATH} is missing: build it with `python -m vit_self_attention_b200.build` "
+        "(nvcc, sm_100a); there is no fallback implementation")
+
+_lib = ctypes.CDLL(LIBRARY_PATH)
+
+_VP = ctypes.c_void_p
+_I = ctypes.c_int
+_lib.vla_attn_fwd.argtypes = [_VP, _VP, _VP, _VP, _I, _I, _I, _I, ctypes.c_float, _VP]
+_lib.vla_attn_fwd.restype = _I
+_lib.vla_attn_fwd_host.argtypes = [_VP, _VP, _VP, _VP, _I, _I, _I, _I, ctypes.c_float, _VP]
+_lib.vla_attn_fwd_host.restype = _I
+_lib.vla_attn_strerror.argtypes = [_I]
+_lib.vla_attn_strerror.restype = ctypes.c_char_p
+_lib.vla_attn_last_device_status.argtypes = [_VP, ctypes.POINTER(_I)]
+_lib.vla_attn_last_device_status.restype = _I
+_lib.vla_attn_reset_device_status.argtypes = [_VP]
+_lib.vla_attn_reset_device_status.restype = _I
+_lib.vla_attn_max_tokens.argtypes = [_I]
+_lib.vla_attn_max_tokens.restype = _I
+_lib.vla_attn_launch_count.argtypes = []
+_lib.vla_attn_launch_count.restype = ctypes.c_uint64
+_lib.vla_attn_set_wait_limit_ns.argtypes = [ctypes.c_uint64]
+_lib.vla_attn_set_wait_limit_ns.restype = None
+
+# Status codes of include/vla_attn.h
+OK = 0
+ERR_NULL = -1
+ERR_SHAPE = -2
+ERR_UNSUPPORTED = -3
+ERR_ALIGN = -4
+ERR_SCALE = -5
+ERR_CUDA = -6
+ERR_TIMEOUT = -7
+ERR_DEVICE = -8
+ERR_MEMORY = -9
+
+EXPORTED_SYMBOLS = (
+    "vla_attn_fwd", "vla_attn_fwd_host", "vla_attn_strerror", "vla_attn_last_device_status",
+    "vla_attn_reset_device_status", "vla_attn_max_tokens", "vla_attn_launch_count",
+    "vla_attn_set_wait_limit_ns",
+)
+
+
+class VlaAttnError(RuntimeError):
+    def __init__(self, status: int):
+        self.status = status
+        super().__init__(f"vla_attn status {status}: {vla_attn_strerror(status)}")
+
+
+def _addr(x) -> int | None:
+    if x is None:
+        return None
+    if isinstance(x, int):
+        return x
+    return int(x.data_ptr())
+
+
+def _stream(stream) -> int | None:
+    if stream is None:
+        import torch
+        return int(torch.cuda.current_stream().cuda_stream)
+    if isinstance(stream, int):
+        return stream
+    return int(stream.cuda_stream)
+
+
+def vla_attn_strerror(status: int) -> str:
+    return _lib.vla_attn_strerror(int(status)).decode()
+
+
+def vla_attn_fwd(q, k, v, o, B: int, N: int, H: int, d: int, scale: float, stream=None,
+                 check: bool = True) -> int:
+    """Enqueue the attention kernel.  ``q/k/v/o`` are tensors or raw device addresses
+    (``k = q + H*d``, ``v = q + 2*H*d`` elements into one packed buffer).  Returns the
+    status; raises ``VlaAttnError`` on a non-zero status when ``check``."""
+    st = _lib.vla_attn_fwd(_addr(q), _addr(k), _addr(v), _addr(o), int(B), int(N), int(H),
+                           int(d), float(scale), _stream(stream))
+    if check and st != OK:
+        raise VlaAttnError(st)
+    return st
+
+
+def vla_attn_fwd_host(qkv_host, o_host, qkv_dev, o_dev, B: int, N: int, H: int, d: int,
+                      scale: float, stream=None, check: bool = True) -> int:
+    """Host-buffer variant: H2D copy, kernel, D2H copy, all enqueued on ``stream``."""
+    st = _lib.vla_attn_fwd_host(_addr(qkv_host), _addr(o_host), _addr(qkv_dev), _addr(o_dev),
+                                int(B), int(N), int(H), int(d), float(scale), _stream(stream))
+    if check and st != OK:
+        raise VlaAttnError(st)
+    return st
+
+
+def vla_attn_last_device_status(stream=None) -> tuple[int, int]:
+    """(status, site) of the device-side status word; synchronises ``stream``."""
+    site = _I(0)
+    st = _lib.vla_attn_last_device_status(_stream(stream), ctypes.byref(site))
+    return st, site.value
+
+
+def vla_attn_reset_device_status(stream=None) -> int:
+    return _lib.vla_attn_reset_device_status(_stream(stream))
+
+
+def vla_attn_max_tokens(d: int) -> int:
+    return _lib.vla_attn_max_tokens(int(d))
+
+
+def vla_attn_launch_count() -> int:
+    return int(_lib.vla_attn_launch_count())
+
+
+def vla_attn_set_wait_limit_ns(ns: int) -> None:
+    _lib.vla_attn_set_wait_limit_ns(int(ns))
+
+
+def attention(qkv, scale: float | None = None, out=None, stream=None):
+    """Convenience wrapper for a contiguous bf16 CUDA tensor ``qkv`` of shape
+    ``[B, N, 3, H, d]``; returns ``out`` (allocated by torch if None) ``[B, N, H, d]``."""
+    import torch
+    if qkv.dim() != 5 or qkv.shape[2] != 3:
+        raise ValueError("qkv must have shape [B, N, 3, H, d]")
+    if qkv.dtype != torch.bfloat16 or not qkv.is_cuda or not qkv.is_contiguous():
+        raise ValueError("qkv must be a contiguous bf16 CUDA tensor")
+    B, N, _, H, d = qkv.shape
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if out is None:
+        out = torch.empty((B, N, H, d), dtype=torch.bfloat16, device=qkv.device)
+    base = qkv.data_ptr()
+    step = H * d * 2
+    vla_attn_fwd(base, base + step, base + 2 * step, out, B, N, H, d, scale, stream)
+    return out
+
+
+__all__ = [
+    "LIBRARY_PATH", "EXPORTED_SYMBOLS", "VlaAttnError", "vla_attn_fwd", "vla_attn_fwd_host",
+    "vla_attn_strerror", "vla_attn_last_device_status", "vla_attn_reset_device_status",
+    "vla_attn_max_tokens", "vla_attn_launch_count", "vla_attn_set_wait_limit_ns", "attention",
+]

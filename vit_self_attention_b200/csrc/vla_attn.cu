@@ -1,0 +1,311 @@
+// Host side of the C ABI declared in include/vla_attn.h: argument checks,
+// TMA tensor maps over the packed [B, N, 3, H, d] bf16 QKV buffer, work
+// decomposition and the launch of the sm_100a attention kernel.
+#include "vla_attn.h"
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <atomic>
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "attn_kernel.cuh"
+
+namespace {
+
+constexpr int kMaxTokens = 577;  // 576 patches + CLS: ViT-L/14 at 336 x 336
+constexpr unsigned long long kDefaultWaitLimitNs = 1000000000ull;
+constexpr int kMaxDevices = 64;
+
+std::atomic<uint64_t> g_launches{0};
+std::atomic<unsigned long long> g_wait_limit_ns{0};
+
+struct DriverFns {
+  PFN_cuTensorMapEncodeTiled_v12000 encode = nullptr;
+  PFN_cuPointerGetAttribute_v4000 ptr_attr = nullptr;
+};
+
+const DriverFns& driver_fns() {
+  static DriverFns fns;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q{};
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fns.encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+    fn = nullptr;
+    if (cudaGetDriverEntryPoint("cuPointerGetAttribute", &fn, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fns.ptr_attr = reinterpret_cast<PFN_cuPointerGetAttribute_v4000>(fn);
+  });
+  return fns;
+}
+
+struct DeviceInfo {
+  bool ready = false;
+  bool supported = false;
+  int sm_count = 0;
+  int max_smem_optin = 0;
+  bool attr64 = false;
+  bool attr72 = false;
+};
+
+std::mutex g_dev_mutex;
+DeviceInfo g_dev[kMaxDevices];
+
+int device_info(int dev, DeviceInfo* out) {
+  if (dev < 0 || dev >= kMaxDevices) return VLA_ATTN_ERR_DEVICE;
+  std::lock_guard<std::mutex> lock(g_dev_mutex);
+  DeviceInfo& di = g_dev[dev];
+  if (!di.ready) {
+    int major = 0, minor = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&di.sm_count, cudaDevAttrMultiProcessorCount, dev) !=
+            cudaSuccess ||
+        cudaDeviceGetAttribute(&di.max_smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin,
+                               dev) != cudaSuccess)
+      return VLA_ATTN_ERR_CUDA;
+    di.supported = (major == 10 && minor == 0);
+    di.ready = true;
+  }
+  *out = di;
+  return di.supported ? VLA_ATTN_OK : VLA_ATTN_ERR_DEVICE;
+}
+
+template <int D>
+int ensure_smem_attr(int dev, int max_smem) {
+  std::lock_guard<std::mutex> lock(g_dev_mutex);
+  bool& done = (D == 64) ? g_dev[dev].attr64 : g_dev[dev].attr72;
+  if (!done) {
+    if (cudaFuncSetAttribute(vla::attn_fwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             max_smem) != cudaSuccess)
+      return VLA_ATTN_ERR_CUDA;
+    done = true;
+  }
+  return VLA_ATTN_OK;
+}
+
+// Checks that [p, p + bytes) lies inside one device allocation of `dev`.
+int check_device_range(const DriverFns& fns, const void* p, size_t bytes, int dev,
+                       uintptr_t* range_lo, uintptr_t* range_hi) {
+  if (fns.ptr_attr == nullptr) return VLA_ATTN_ERR_CUDA;
+  const CUdeviceptr dp = reinterpret_cast<CUdeviceptr>(p);
+  unsigned int mem_type = 0;
+  if (fns.ptr_attr(&mem_type, CU_POINTER_ATTRIBUTE_MEMORY_TYPE, dp) != CUDA_SUCCESS ||
+      mem_type != CU_MEMORYTYPE_DEVICE)
+    return VLA_ATTN_ERR_MEMORY;
+  int ordinal = -1;
+  if (fns.ptr_attr(&ordinal, CU_POINTER_ATTRIBUTE_DEVICE_ORDINAL, dp) != CUDA_SUCCESS ||
+      ordinal != dev)
+    return VLA_ATTN_ERR_MEMORY;
+  CUdeviceptr start = 0;
+  size_t size = 0;
+  if (fns.ptr_attr(&start, CU_POINTER_ATTRIBUTE_RANGE_START_ADDR, dp) != CUDA_SUCCESS ||
+      fns.ptr_attr(&size, CU_POINTER_ATTRIBUTE_RANGE_SIZE, dp) != CUDA_SUCCESS)
+    return VLA_ATTN_ERR_MEMORY;
+  const uintptr_t lo = static_cast<uintptr_t>(dp);
+  if (lo < start || bytes > size || lo - start > size - bytes) return VLA_ATTN_ERR_MEMORY;
+  *range_lo = lo;
+  *range_hi = lo + bytes;
+  return VLA_ATTN_OK;
+}
+
+int encode_map(const DriverFns& fns, CUtensorMap* map, const void* qkv, int B, int N, int H,
+               int d, uint32_t box_c, CUtensorMapSwizzle swizzle) {
+  const cuuint64_t dims[5] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(H), 3u,
+                              static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(B)};
+  const cuuint64_t tok = 3ull * H * d * 2ull;
+  const cuuint64_t strides[4] = {static_cast<cuuint64_t>(d) * 2ull,
+                                 static_cast<cuuint64_t>(H) * d * 2ull, tok,
+                                 tok * static_cast<cuuint64_t>(N)};
+  const cuuint32_t box[5] = {box_c, 1u, 1u, static_cast<cuuint32_t>(vla::kTileRows), 1u};
+  const cuuint32_t elem_strides[5] = {1u, 1u, 1u, 1u, 1u};
+  const CUresult rc = fns.encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void*>(qkv),
+                                 dims, strides, box, elem_strides, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                                 swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                                 CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return rc == CUDA_SUCCESS ? VLA_ATTN_OK : VLA_ATTN_ERR_CUDA;
+}
+
+int check_args(const void* q, const void* k, const void* v, const void* o, int B, int N, int H,
+               int d, float scale) {
+  if (q == nullptr || k == nullptr || v == nullptr || o == nullptr) return VLA_ATTN_ERR_NULL;
+  if (B < 1 || N < 1 || H < 1) return VLA_ATTN_ERR_SHAPE;
+  if (d != 64 && d != 72) return VLA_ATTN_ERR_UNSUPPORTED;
+  if (N > kMaxTokens) return VLA_ATTN_ERR_UNSUPPORTED;
+  const uintptr_t qa = reinterpret_cast<uintptr_t>(q);
+  const uintptr_t hd_bytes = static_cast<uintptr_t>(H) * d * 2u;
+  if (reinterpret_cast<uintptr_t>(k) != qa + hd_bytes ||
+      reinterpret_cast<uintptr_t>(v) != qa + 2u * hd_bytes)
+    return VLA_ATTN_ERR_SHAPE;
+  if ((qa & 15u) != 0 || (reinterpret_cast<uintptr_t>(o) & 15u) != 0) return VLA_ATTN_ERR_ALIGN;
+  if (!std::isfinite(scale) || !(scale > 0.0f)) return VLA_ATTN_ERR_SCALE;
+  // TMA extents are 32-bit per dimension; element counts must fit size_t math below.
+  const unsigned long long total = 3ull * B * N * H * d;
+  if (total > (1ull << 46)) return VLA_ATTN_ERR_SHAPE;
+  return VLA_ATTN_OK;
+}
+
+template <int D>
+int launch(const void* q, void* o, int B, int N, int H, float scale, cudaStream_t stream,
+           const DeviceInfo& di, int dev, const DriverFns& fns) {
+  constexpr uint32_t kTile = vla::TileGeom<D>::kBytes;
+  vla::AttnParams prm;
+  std::memset(&prm, 0, sizeof(prm));
+  int rc = encode_map(fns, &prm.tm_main, q, B, N, H, D, 64u, CU_TENSOR_MAP_SWIZZLE_128B);
+  if (rc != VLA_ATTN_OK) return rc;
+  if (D > 64) {
+    rc = encode_map(fns, &prm.tm_tail, q, B, N, H, D, 16u, CU_TENSOR_MAP_SWIZZLE_32B);
+    if (rc != VLA_ATTN_OK) return rc;
+  }
+  const int nb = (N + vla::kTileRows - 1) / vla::kTileRows;
+  const int max_smem = di.max_smem_optin;
+  int ring = (max_smem - static_cast<int>(2 * kTile + vla::kBarrierRegionBytes + vla::kAlignSlack)) /
+             static_cast<int>(2 * kTile);
+  if (ring > vla::kMaxRing) ring = vla::kMaxRing;
+  if (ring < 2) return VLA_ATTN_ERR_DEVICE;
+  const uint32_t smem = vla::smem_bytes_for_ring<D>(ring);
+
+  prm.o = static_cast<__nv_bfloat16*>(o);
+  prm.B = B;
+  prm.N = N;
+  prm.H = H;
+  prm.num_kblocks = nb;
+  prm.num_qtiles = nb;
+  prm.rounds_per_head = (nb + 1) / 2;
+  const long long heads = static_cast<long long>(B) * H;
+  prm.rounds_per_unit = heads >= di.sm_count ? prm.rounds_per_head : 1;
+  prm.units_per_head = prm.rounds_per_head / prm.rounds_per_unit;
+  const long long units = heads * prm.units_per_head;
+  if (units > 0x7FFFFFFFll) return VLA_ATTN_ERR_SHAPE;
+  prm.num_units = static_cast<int>(units);
+  prm.ring = ring;
+  prm.reuse = nb <= ring ? 1 : 0;
+  prm.c = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
+  const unsigned long long lim = g_wait_limit_ns.load();
+  prm.wait_limit_ns = lim == 0 ? kDefaultWaitLimitNs : lim;
+
+  rc = ensure_smem_attr<D>(dev, max_smem);
+  if (rc != VLA_ATTN_OK) return rc;
+
+  const int grid = static_cast<int>(units < di.sm_count ? units : di.sm_count);
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(static_cast<unsigned>(grid), 1, 1);
+  cfg.blockDim = dim3(vla::kThreads, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cfg.attrs = nullptr;
+  cfg.numAttrs = 0;
+  if (cudaLaunchKernelEx(&cfg, vla::attn_fwd_kernel<D>, prm) != cudaSuccess) {
+    (void)cudaGetLastError();
+    return VLA_ATTN_ERR_CUDA;
+  }
+  g_launches.fetch_add(1);
+  return VLA_ATTN_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int vla_attn_fwd(const void* q, const void* k, const void* v, void* o, int B, int N, int H,
+                 int d, float scale, void* stream) {
+  int rc = check_args(q, k, v, o, B, N, H, d, scale);
+  if (rc != VLA_ATTN_OK) return rc;
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) return VLA_ATTN_ERR_CUDA;
+  DeviceInfo di;
+  rc = device_info(dev, &di);
+  if (rc != VLA_ATTN_OK) return rc;
+  const DriverFns& fns = driver_fns();
+  if (fns.encode == nullptr || fns.ptr_attr == nullptr) return VLA_ATTN_ERR_CUDA;
+  const size_t in_bytes = 3ull * B * N * H * d * 2ull;
+  const size_t out_bytes = 1ull * B * N * H * d * 2ull;
+  uintptr_t in_lo = 0, in_hi = 0, out_lo = 0, out_hi = 0;
+  rc = check_device_range(fns, q, in_bytes, dev, &in_lo, &in_hi);
+  if (rc != VLA_ATTN_OK) return rc;
+  rc = check_device_range(fns, o, out_bytes, dev, &out_lo, &out_hi);
+  if (rc != VLA_ATTN_OK) return rc;
+  if (out_lo < in_hi && in_lo < out_hi) return VLA_ATTN_ERR_MEMORY;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (d == 64) return launch<64>(q, o, B, N, H, scale, st, di, dev, fns);
+  return launch<72>(q, o, B, N, H, scale, st, di, dev, fns);
+}
+
+int vla_attn_fwd_host(const void* qkv_host, void* o_host, void* qkv_dev, void* o_dev, int B,
+                      int N, int H, int d, float scale, void* stream) {
+  if (qkv_host == nullptr || o_host == nullptr || qkv_dev == nullptr || o_dev == nullptr)
+    return VLA_ATTN_ERR_NULL;
+  const char* qd = static_cast<const char*>(qkv_dev);
+  const size_t hd_bytes = static_cast<size_t>(H > 0 ? H : 0) * (d > 0 ? d : 0) * 2u;
+  int rc = check_args(qd, qd + hd_bytes, qd + 2 * hd_bytes, o_dev, B, N, H, d, scale);
+  if (rc != VLA_ATTN_OK) return rc;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const size_t in_bytes = 3ull * B * N * H * d * 2ull;
+  const size_t out_bytes = 1ull * B * N * H * d * 2ull;
+  if (cudaMemcpyAsync(qkv_dev, qkv_host, in_bytes, cudaMemcpyHostToDevice, st) != cudaSuccess)
+    return VLA_ATTN_ERR_CUDA;
+  rc = vla_attn_fwd(qd, qd + hd_bytes, qd + 2 * hd_bytes, o_dev, B, N, H, d, scale, stream);
+  if (rc != VLA_ATTN_OK) return rc;
+  if (cudaMemcpyAsync(o_host, o_dev, out_bytes, cudaMemcpyDeviceToHost, st) != cudaSuccess)
+    return VLA_ATTN_ERR_CUDA;
+  return VLA_ATTN_OK;
+}
+
+const char* vla_attn_strerror(int status) {
+  switch (status) {
+    case VLA_ATTN_OK: return "ok";
+    case VLA_ATTN_ERR_NULL: return "a required pointer is NULL";
+    case VLA_ATTN_ERR_SHAPE:
+      return "bad shape: B, N, H must be >= 1 and q/k/v must point into one packed [B,N,3,H,d] "
+             "buffer (k = q + H*d, v = q + 2*H*d elements)";
+    case VLA_ATTN_ERR_UNSUPPORTED:
+      return "unsupported: head dimension must be 64 or 72 and N at most 577";
+    case VLA_ATTN_ERR_ALIGN: return "q and o must be 16-byte aligned";
+    case VLA_ATTN_ERR_SCALE: return "scale must be finite and > 0";
+    case VLA_ATTN_ERR_CUDA: return "a CUDA runtime or driver call failed";
+    case VLA_ATTN_ERR_TIMEOUT: return "a bounded wait inside the attention kernel ran out";
+    case VLA_ATTN_ERR_DEVICE: return "the current device is not an sm_100 (B200-class) GPU";
+    case VLA_ATTN_ERR_MEMORY:
+      return "a pointer is not device memory of the current device, its allocation is too "
+             "small for the shape, or the output overlaps the input";
+    default: return "unknown vla_attn status";
+  }
+}
+
+int vla_attn_last_device_status(void* stream, int* site) {
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  int word = 0;
+  if (cudaMemcpyFromSymbolAsync(&word, vla::g_vla_attn_status, sizeof(int), 0,
+                                cudaMemcpyDeviceToHost, st) != cudaSuccess)
+    return VLA_ATTN_ERR_CUDA;
+  if (cudaStreamSynchronize(st) != cudaSuccess) return VLA_ATTN_ERR_CUDA;
+  if (site != nullptr) *site = word == 0 ? 0 : word - 1000;
+  return word == 0 ? VLA_ATTN_OK : VLA_ATTN_ERR_TIMEOUT;
+}
+
+int vla_attn_reset_device_status(void* stream) {
+  static const int zero = 0;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (cudaMemcpyToSymbolAsync(vla::g_vla_attn_status, &zero, sizeof(int), 0,
+                              cudaMemcpyHostToDevice, st) != cudaSuccess)
+    return VLA_ATTN_ERR_CUDA;
+  if (cudaStreamSynchronize(st) != cudaSuccess) return VLA_ATTN_ERR_CUDA;
+  return VLA_ATTN_OK;
+}
+
+int vla_attn_max_tokens(int d) { return (d == 64 || d == 72) ? kMaxTokens : 0; }
+
+uint64_t vla_attn_launch_count(void) { return g_launches.load(); }
+
+void vla_attn_set_wait_limit_ns(uint64_t ns) { g_wait_limit_ns.store(ns); }
+
+}  // extern "C"
