@@ -15,6 +15,7 @@ bounded sample of the same workload (rank 0 only).
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import glob
 import hashlib
 import json
@@ -212,6 +213,8 @@ def run_ours(args, rank: int, world: int, local_rank: int) -> None:
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
     c = WORKLOAD
+    if args.images is not None:
+        c = dataclasses.replace(c, B=int(args.images), name=f"{c.name}_B{int(args.images)}")
     stream = torch.cuda.current_stream(dev)
 
     bits = si.packed_qkv(c.B, c.N, c.H, c.d, c.seed(0) + 7919 * rank)
@@ -252,28 +255,30 @@ def run_ours(args, rank: int, world: int, local_rank: int) -> None:
         raise RuntimeError(f"device status {st} (site {site}) after the timed region")
 
     # ---- end-to-end through the host-buffer C-ABI entry (pinned host memory)
-    host_out = torch.empty((c.B, c.N, c.H, c.d), dtype=torch.int16).pin_memory()
-    dev_in = torch.empty(bits.shape, dtype=torch.int16, device=dev)
-    dev_out = torch.empty((c.B, c.N, c.H, c.d), dtype=torch.int16, device=dev)
     e2e_steps = max(2, min(args.steps, 10))
+    e2e_ms = float("nan")
+    if not args.no_e2e:
+        host_out = torch.empty((c.B, c.N, c.H, c.d), dtype=torch.int16).pin_memory()
+        dev_in = torch.empty(bits.shape, dtype=torch.int16, device=dev)
+        dev_out = torch.empty((c.B, c.N, c.H, c.d), dtype=torch.int16, device=dev)
 
-    def e2e_step():
-        vab.vla_attn_fwd_host(host_in, host_out, dev_in, dev_out, c.B, c.N, c.H, c.d, c.scale,
-                              stream)
+        def e2e_step():
+            vab.vla_attn_fwd_host(host_in, host_out, dev_in, dev_out, c.B, c.N, c.H, c.d,
+                                  c.scale, stream)
 
-    e2e_step()
-    torch.cuda.synchronize()
-    barrier()
-    torch.cuda.synchronize()
-    e0 = torch.cuda.Event(enable_timing=True)
-    e1 = torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(e2e_steps):
         e2e_step()
-    e1.record(stream)
-    torch.cuda.synchronize()
-    barrier()
-    e2e_ms = e0.elapsed_time(e1)
+        torch.cuda.synchronize()
+        barrier()
+        torch.cuda.synchronize()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(e2e_steps):
+            e2e_step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        e2e_ms = e0.elapsed_time(e1)
 
     if world > 1:
         t = torch.tensor([ms, e2e_ms], dtype=torch.float64, device=dev)
@@ -311,10 +316,11 @@ def run_ours(args, rank: int, world: int, local_rank: int) -> None:
                      "hbm_gbs_achieved": c.bytes() / (ms_step / 1e3) / 1e9,
                      "traffic_source": traffic_src},
         "cpu_baseline": cpu,
-        "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": int(bits.nbytes),
-                "d2h_bytes_per_step": int(c.B * c.N * c.H * c.d * 2),
-                "steps": e2e_steps, "ms_per_step": e2e_ms / e2e_steps,
-                "api": "vla_attn_fwd_host (pinned host buffers)"},
+        "e2e": None if args.no_e2e else {
+            "value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": int(bits.nbytes),
+            "d2h_bytes_per_step": int(c.B * c.N * c.H * c.d * 2),
+            "steps": e2e_steps, "ms_per_step": e2e_ms / e2e_steps,
+            "api": "vla_attn_fwd_host (pinned host buffers)"},
         "gpu_launches": int(launches),
         "clocks": clocks.summary(),
         "kernel_source_sha256_16": kernel_source_hash(),
@@ -331,6 +337,9 @@ def main() -> None:
     ap.add_argument("--cpu-seconds", type=float, default=10.0,
                     help="target duration of the CPU oracle baseline sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end leg")
+    ap.add_argument("--images", type=int, default=None,
+                    help="override B (profiling captures of a smaller case of the same kernel)")
     args = ap.parse_args()
 
     world = int(os.environ.get("WORLD_SIZE", "1"))

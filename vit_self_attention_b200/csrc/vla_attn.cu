@@ -53,8 +53,8 @@ struct DeviceInfo {
   bool supported = false;
   int sm_count = 0;
   int max_smem_optin = 0;
-  bool attr64 = false;
-  bool attr72 = false;
+  int attr64 = 0;  // dynamic shared memory limit set on the d = 64 kernel (0 = not yet)
+  int attr72 = 0;
 };
 
 std::mutex g_dev_mutex;
@@ -80,17 +80,31 @@ int device_info(int dev, DeviceInfo* out) {
   return di.supported ? VLA_ATTN_OK : VLA_ATTN_ERR_DEVICE;
 }
 
+// Raises the kernel's dynamic shared-memory limit to at least `smem` bytes.
 template <int D>
-int ensure_smem_attr(int dev, int max_smem) {
+int ensure_smem_attr(int dev, int smem) {
   std::lock_guard<std::mutex> lock(g_dev_mutex);
-  bool& done = (D == 64) ? g_dev[dev].attr64 : g_dev[dev].attr72;
-  if (!done) {
+  int& cur = (D == 64) ? g_dev[dev].attr64 : g_dev[dev].attr72;
+  if (cur < smem) {
     if (cudaFuncSetAttribute(vla::attn_fwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             max_smem) != cudaSuccess)
+                             smem) != cudaSuccess)
       return VLA_ATTN_ERR_CUDA;
-    done = true;
+    cur = smem;
   }
   return VLA_ATTN_OK;
+}
+
+// Static shared memory of the kernel instantiation (0 for the product build).
+template <int D>
+int static_smem_bytes() {
+  static int bytes = -1;
+  if (bytes < 0) {
+    cudaFuncAttributes fa{};
+    bytes = cudaFuncGetAttributes(&fa, vla::attn_fwd_kernel<D>) == cudaSuccess
+                ? static_cast<int>(fa.sharedSizeBytes)
+                : 0;
+  }
+  return bytes;
 }
 
 // Checks that [p, p + bytes) lies inside one device allocation of `dev`.
@@ -167,7 +181,7 @@ int launch(const void* q, void* o, int B, int N, int H, float scale, cudaStream_
     if (rc != VLA_ATTN_OK) return rc;
   }
   const int nb = (N + vla::kTileRows - 1) / vla::kTileRows;
-  const int max_smem = di.max_smem_optin;
+  const int max_smem = di.max_smem_optin - static_smem_bytes<D>();
   int ring = (max_smem - static_cast<int>(2 * kTile + vla::kBarrierRegionBytes + vla::kAlignSlack)) /
              static_cast<int>(2 * kTile);
   if (ring > vla::kMaxRing) ring = vla::kMaxRing;
@@ -193,7 +207,7 @@ int launch(const void* q, void* o, int B, int N, int H, float scale, cudaStream_
   const unsigned long long lim = g_wait_limit_ns.load();
   prm.wait_limit_ns = lim == 0 ? kDefaultWaitLimitNs : lim;
 
-  rc = ensure_smem_attr<D>(dev, max_smem);
+  rc = ensure_smem_attr<D>(dev, static_cast<int>(smem));
   if (rc != VLA_ATTN_OK) return rc;
 
   const int grid = static_cast<int>(units < di.sm_count ? units : di.sm_count);
