@@ -26,14 +26,15 @@ def test_configs_every_call(cfg):
         assert_parity(got, want, f"config {cfg} ({c.name}) call {call}")
 
 
-EDGE_N = [1, 2, 15, 16, 17, 63, 64, 65, 127, 128, 129, 200, 255, 256, 257, 383, 384, 385, 511,
-          512, 513, 576, 577]
+# Boundaries of 128-row query tiles / 128-key blocks (d=64) and 112-key blocks (d=72).
+EDGE_N = [1, 2, 15, 16, 17, 63, 64, 65, 111, 112, 113, 127, 128, 129, 200, 224, 225, 255, 256,
+          257, 336, 337, 383, 384, 385, 448, 449, 511, 512, 513, 560, 561, 576, 577]
 
 
 @pytest.mark.parametrize("d", [64, 72])
 @pytest.mark.parametrize("N", EDGE_N)
 def test_edge_token_counts(N, d):
-    """Ragged query tiles and key blocks, single- and two-slot rounds, ring streaming (d=72, N>512)."""
+    """Ragged query tiles and key blocks, single- and two-slot rounds, ring streaming (d=72, N>560)."""
     B, H = 2, 3
     bits = si.packed_qkv(B, N, H, d, seed=70000 + 10 * N + d)
     scale = 1.0 / math.sqrt(d)

@@ -10,46 +10,47 @@
 //
 // Blackwell mapping (one persistent CTA per SM, 384 threads = 3 warpgroups):
 //   warp 9      TMA producer: Q tiles (128 query rows) into two Q slots, K and
-//               V blocks (128 keys) into a ring of `ring` slots.  With
-//               `reuse`, a head's K/V blocks are loaded once and serve all of
-//               that head's Q tiles.
+//               V blocks (BK keys) into a ring of `ring` slots.  With `reuse`,
+//               a head's K/V blocks are loaded once and serve all of that
+//               head's Q tiles.
 //   warp 8      tcgen05 issuer (one thread): S = Q K^T into tensor memory
-//               (SS MMA, M=128, N=keys of the block, K=16 steps over d), then
-//               O += P V with P read from tensor memory (TS MMA, N=64 or
-//               64+16).
+//               (SS MMA, M=128, N=keys of the block, K=16 steps over d) and
+//               O += P V with P read from tensor memory (TS MMA, N=64, plus
+//               N=16 for d=72).
 //   warps 0-7   softmax, one warpgroup per Q slot, one thread per query row
 //               (= tensor-memory lane): online softmax in fp32 with exp2 and a
-//               pre-scaled log2(e), P packed to bf16 pairs and stored back over
-//               its own S columns, O rescaled in tensor memory only when the
-//               running maximum grows by more than 2^8, epilogue O / l -> bf16
-//               with 16-byte stores.
+//               pre-scaled log2(e), P as bf16 pairs in its own tensor-memory
+//               columns, O rescaled in tensor memory only when the running
+//               maximum grows by more than 2^8, epilogue O / l -> bf16 with
+//               16-byte stores.
 //   warps 10-11 idle.
 //
-// Work is a sequence of rounds.  A full round holds two Q tiles of one head:
-// slot s owns S buffer s and O accumulator s, the tensor core works on one
-// slot while the other slot's softmax runs, and the two softmax warpgroups
-// take turns on the exp2 unit (an mbarrier token passed back and forth), so
-// the special-function pipe stays busy instead of both groups stalling on it
-// at once.  A half round (the odd last tile of a head) has only slot 0; it
-// then uses both S buffers in turn so S of the next key block is computed
-// while the current one is being exponentiated.
+// Pipelining.  A softmax thread signals "S consumed" as soon as it has the S
+// row of block j in registers, so the tensor core computes S of block j+1
+// while block j is being exponentiated; P V of block j follows as soon as P
+// is stored.  A full round holds two Q tiles of one head (slots 0 and 1, one
+// per softmax warpgroup) and the two warpgroups take turns on the exp2 unit
+// (an mbarrier token passed back and forth) so the special-function pipe is
+// never contended by both at once.  A half round (the odd last tile of a
+// head) has slot 0 only.
 //
-// Tensor memory (512 columns): S buffer b at columns [256 b, 256 b + 128)
-// (fp32; overwritten in place by P as bf16 pairs in its first 64 columns);
-// O accumulator s at [256 s + 128, 256 s + 128 + 80).
+// Tensor memory (512 columns): slot s owns columns [256 s, 256 s + 256):
+// S at +0 (BK fp32 columns), O at +BK (DP = 64 or 80 fp32 columns), P at
+// +BK+DP (BK/2 columns of bf16 pairs).  d=64 uses BK=128 (128+64+64 = 256),
+// d=72 uses BK=112 (112+80+56 = 248).
 //
-// Shared memory per 128-row tile: channels 0..63 as a 128-byte-swizzled
-// 128 x 128 B region (TMA box {64,1,1,128,1}); for d = 72 the channels 64..79
-// (72..79 zero-filled by TMA) as a 32-byte-swizzled 128 x 32 B region.
-// Q and K are read K-major by the MMA, V MN-major.
+// Shared memory: a tile row holds channels 0..63 in a 128-byte-swizzled
+// region (TMA box {64,1,1,rows,1}); for d=72 channels 64..79 (72..79
+// zero-filled by TMA) sit in a 32-byte-swizzled region.  Q and K are read
+// K-major by the MMA, V MN-major.
 //
 // Every mbarrier wait is bounded; a wait that runs out sets a shared abort
 // flag and the device status word, every role then leaves its loop, the
 // producer waits (bounded) for its own TMA copies, the MMA thread waits
 // (bounded) for its own tensor-core work, and the tensor memory is freed.
-// Each barrier is waited on in phase order by every thread that waits on it,
-// or it cannot complete twice without an intervening wait, so a parity wait
-// never confuses two phases.
+// Every barrier has one consumer role that waits on each of its phases in
+// order, and no barrier can complete twice before its consumer has waited,
+// so a parity wait never confuses two phases.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -59,34 +60,33 @@
 
 namespace vla {
 
-constexpr int kTileRows = 128;  // query rows per tile = keys per block = TMEM lanes
+constexpr int kQRows = 128;  // query rows per tile = TMEM lanes = MMA M
 constexpr int kMmaWarp = 8;
 constexpr int kLoadWarp = 9;
 constexpr int kThreads = 384;
 constexpr int kMaxRing = 6;
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kMainRegionBytes = 128 * 128;  // 128 rows x 64 bf16 channels
-constexpr uint32_t kTailRegionBytes = 128 * 32;   // 128 rows x 16 bf16 channels
 constexpr int kNumBarriers = 14 + 4 * kMaxRing + 1;
-constexpr uint32_t kBarrierRegionBytes = 512;     // barriers + tmem address + abort flag
+constexpr uint32_t kBarrierRegionBytes = 512;  // barriers + tmem address + abort flag
 constexpr uint32_t kAlignSlack = 1024;
 constexpr unsigned long long kDrainLimitNs = 100000000ull;
 
 // Device status codes (the first wait that ran out records its site).
 enum : int {
   kSiteLoadQ = 1, kSiteLoadK = 2, kSiteLoadV = 3,
-  kSiteMmaQ = 11, kSiteMmaK = 12, kSiteMmaV = 13, kSiteMmaP = 14,
+  kSiteMmaQ = 11, kSiteMmaK = 12, kSiteMmaV = 13, kSiteMmaP = 14, kSiteMmaFree = 15,
   kSiteSoftS = 21, kSiteSoftO = 22, kSiteSoftTok = 23,
   kSiteDrain = 31,
 };
 
 __device__ int g_vla_attn_status;  // 0 = ok, else 1000 + site of the first timed-out wait
 
-// Timeline hook for diagnostic builds: a translation unit may define
-// VLA_TRACE_EVENT(kind, slot, block) before including this header to record
-// when each role reaches the points below; by default it compiles to nothing.
+// Timeline hooks for diagnostic builds: a translation unit may define these
+// before including this header to record when each role reaches the points
+// below; by default they compile to nothing.
 enum : int {
-  kTrMmaS = 1, kTrMmaPV = 2,
+  kTrMmaS = 1, kTrMmaPV = 2, kTrMmaSDone = 3, kTrMmaPVDone = 4, kTrMmaFree = 5, kTrMmaP = 6,
+  kTrMmaV = 7, kTrMmaK = 8,
   kTrSoftS = 10, kTrSoftMax = 11, kTrSoftTok = 12, kTrSoftExp = 13, kTrSoftP = 14,
   kTrSoftEpi = 15,
 };
@@ -98,46 +98,59 @@ enum : int {
 #endif
 
 template <int D>
-struct TileGeom {
+struct Geom {
   static_assert(D == 64 || D == 72, "head dimension must be 64 or 72");
   static constexpr bool kHasTail = D > 64;
-  static constexpr uint32_t kBytes = kMainRegionBytes + (kHasTail ? kTailRegionBytes : 0);
+  static constexpr int BK = kHasTail ? 112 : 128;  // keys per block
+  static constexpr int DP = kHasTail ? 80 : 64;    // MMA N of P V (d padded to 16)
+  // Q tile: 128 rows x 128 B (SW128) [+ 128 rows x 32 B (SW32)].
+  static constexpr uint32_t kQTail = 128 * 128;
+  static constexpr uint32_t kQBytes = kQTail + (kHasTail ? 128 * 32 : 0);
+  // K / V block: BK rows x 128 B (SW128) [+ BK rows x 32 B (SW32)], stride a
+  // multiple of 1024 B so every region keeps its swizzle alignment.
+  static constexpr uint32_t kKVTail = BK * 128;
+  static constexpr uint32_t kKVBytes = kKVTail + (kHasTail ? BK * 32 : 0);
+  static constexpr uint32_t kKVStride = (kKVBytes + 1023u) & ~1023u;
+  // Tensor-memory columns within a slot.
+  static constexpr uint32_t kColO = BK;
+  static constexpr uint32_t kColP = BK + DP;
+  static_assert(BK + DP + BK / 2 <= 256, "slot does not fit its 256 TMEM columns");
 };
 
 struct AttnParams {
-  CUtensorMap tm_main;  // 128B-swizzled box {64, 1, 1, 128, 1} over the packed QKV
-  CUtensorMap tm_tail;  // 32B-swizzled box {16, 1, 1, 128, 1}, channels 64..79 (d = 72)
-  __nv_bfloat16* o;     // [B, N, H, d]
+  CUtensorMap tm_q;        // 128B-swizzled box {64, 1, 1, 128, 1} (Q tiles)
+  CUtensorMap tm_q_tail;   // 32B-swizzled box {16, 1, 1, 128, 1}, channels 64..79 (d = 72)
+  CUtensorMap tm_kv;       // 128B-swizzled box {64, 1, 1, BK, 1} (K / V blocks)
+  CUtensorMap tm_kv_tail;  // 32B-swizzled box {16, 1, 1, BK, 1} (d = 72)
+  __nv_bfloat16* o;        // [B, N, H, d]
   int B, N, H;
-  int num_kblocks;      // ceil(N / 128)
-  int num_qtiles;       // ceil(N / 128)
-  int rounds_per_head;  // ceil(num_qtiles / 2): a round = up to two Q tiles
-  int rounds_per_unit;  // rounds_per_head (whole head) or 1
+  int num_kblocks;         // ceil(N / BK)
+  int num_qtiles;          // ceil(N / 128)
+  int rounds_per_head;     // ceil(num_qtiles / 2): a round = up to two Q tiles
+  int rounds_per_unit;     // rounds_per_head (whole head) or 1
   int units_per_head;
   int num_units;
-  int ring;             // K/V ring slots (<= kMaxRing)
-  int reuse;            // 1 when num_kblocks <= ring: a unit loads its K/V once
-  float c;              // scale * log2(e)
+  int ring;                // K/V ring slots (<= kMaxRing)
+  int reuse;               // 1 when num_kblocks <= ring: a unit loads its K/V once
+  float c;                 // scale * log2(e)
   unsigned long long wait_limit_ns;
 };
 
 template <int D>
 __host__ __device__ constexpr uint32_t smem_bytes_for_ring(int ring) {
-  return (2u + 2u * static_cast<uint32_t>(ring)) * TileGeom<D>::kBytes + kBarrierRegionBytes +
-         kAlignSlack;
+  return 2u * Geom<D>::kQBytes + 2u * static_cast<uint32_t>(ring) * Geom<D>::kKVStride +
+         kBarrierRegionBytes + kAlignSlack;
 }
 
 struct Barriers {
   uint32_t base;
   __device__ uint32_t q_full(int s) const { return base + 8u * (0 + s); }
   __device__ uint32_t q_empty(int s) const { return base + 8u * (2 + s); }
-  // S ready / P ready, per "channel": 0 = buffer 0 (slot 0), 1 = buffer 1 used
-  // by slot 1 in full rounds, 2 = buffer 1 used by slot 0 in half rounds.
-  // Each channel has exactly one consumer warpgroup, which waits on every phase.
-  __device__ uint32_t s_full(int ch) const { return base + 8u * (4 + ch); }
-  __device__ uint32_t p_full(int ch) const { return base + 8u * (7 + ch); }
-  __device__ uint32_t o_prog(int s) const { return base + 8u * (10 + s); }  // per O slot, every PV
-  __device__ uint32_t tok(int s) const { return base + 8u * (12 + s); }     // exp2 turn of slot s
+  __device__ uint32_t s_full(int s) const { return base + 8u * (4 + s); }   // S in TMEM
+  __device__ uint32_t s_free(int s) const { return base + 8u * (6 + s); }   // S read out
+  __device__ uint32_t p_full(int s) const { return base + 8u * (8 + s); }   // P in TMEM
+  __device__ uint32_t o_prog(int s) const { return base + 8u * (10 + s); }  // each P V done
+  __device__ uint32_t tok(int s) const { return base + 8u * (12 + s); }     // exp2 turn
   __device__ uint32_t k_full(int i) const { return base + 8u * (14 + i); }
   __device__ uint32_t k_empty(int i) const { return base + 8u * (14 + kMaxRing + i); }
   __device__ uint32_t v_full(int i) const { return base + 8u * (14 + 2 * kMaxRing + i); }
@@ -145,22 +158,30 @@ struct Barriers {
   __device__ uint32_t drain() const { return base + 8u * (14 + 4 * kMaxRing); }
 };
 
-// Bounded wait for the phase of `bar` with the given parity.  Returns false
+// Bounded wait for the phase of `bar` with the given parity, executed by a
+// whole converged warp; the result is the same in every lane.  Returns false
 // when the CTA has aborted or this wait ran out (which aborts the CTA).
 __device__ __forceinline__ bool wait_bounded(uint32_t bar, uint32_t parity,
                                              volatile int* abort_flag,
                                              unsigned long long limit_ns, int site) {
-  if (mbar_try_wait(bar, parity)) return true;
-  const uint64_t t0 = global_timer_ns();
-  while (true) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if (*abort_flag) return false;
-    if (global_timer_ns() - t0 > limit_ns) {
-      *abort_flag = 1;
-      atomicCAS(&g_vla_attn_status, 0, 1000 + site);
-      return false;
+  bool done = mbar_try_wait(bar, parity);
+  if (__all_sync(0xffffffffu, done)) return true;
+  if (!done) {
+    const uint64_t t0 = global_timer_ns();
+    while (true) {
+      if (mbar_try_wait(bar, parity)) {
+        done = true;
+        break;
+      }
+      if (*abort_flag) break;
+      if (global_timer_ns() - t0 > limit_ns) {
+        *abort_flag = 1;
+        atomicCAS(&g_vla_attn_status, 0, 1000 + site);
+        break;
+      }
     }
   }
+  return __all_sync(0xffffffffu, done);
 }
 
 // Wait used while draining: ignores the abort flag, gives up after limit_ns.
@@ -175,18 +196,20 @@ __device__ __forceinline__ void wait_drain(uint32_t bar, uint32_t parity,
   }
 }
 
+// Keys of block j rounded up to the MMA granularity of 16.
+template <int BK>
 __device__ __forceinline__ int block_cols(int N, int j) {
-  const int rem = N - j * kTileRows;
+  const int rem = N - j * BK;
   const int n16 = (rem + 15) & ~15;
-  return n16 < kTileRows ? n16 : kTileRows;
+  return n16 < BK ? n16 : BK;
 }
 
 // One (unit, round) step of the schedule, identical for every role.
 struct Round {
-  int b, h, r;      // image, head, round index within the head
-  int nslots;       // 2 = full round (tiles 2r, 2r+1), 1 = half round (tile 2r only)
-  bool first;       // first round of its unit
-  bool last;        // last round of its unit
+  int b, h, r;  // image, head, round index within the head
+  int nslots;   // 2 = full round (tiles 2r, 2r+1), 1 = half round (tile 2r only)
+  bool first;   // first round of its unit
+  bool last;    // last round of its unit
 };
 
 __device__ __forceinline__ Round make_round(const AttnParams& p, int u, int rr) {
@@ -201,30 +224,56 @@ __device__ __forceinline__ Round make_round(const AttnParams& p, int u, int rr) 
   return x;
 }
 
+// Position of a K/V load event in the ring: slot index and the parity of
+// the number of times the ring has wrapped (the phase its barriers are in).
+struct RingPos {
+  int slot;
+  uint32_t phase;
+  __device__ __forceinline__ void advance(int R) {
+    if (++slot == R) {
+      slot = 0;
+      phase ^= 1u;
+    }
+  }
+};
+
 // ------------------------------------------------------------ producer
 template <int D>
 __device__ void load_role(const AttnParams& p, uint32_t sQ, uint32_t sK, uint32_t sV,
                           const Barriers& bar, volatile int* abort_flag) {
-  constexpr uint32_t kTile = TileGeom<D>::kBytes;
+  using G = Geom<D>;
   const int R = p.ring;
   const int nb = p.num_kblocks;
   uint32_t nq0 = 0, nq1 = 0;  // Q loads issued into slot 0 / 1
   uint32_t kv_ev = 0;         // K/V load events issued
+  RingPos pos{0, 0u};         // ring position of the next K/V event
   bool ok = true;
 
-  auto load_tile = [&](uint32_t dst, uint32_t mbar, int w, int row0, int b, int h) {
-    tma_load_5d(dst, &p.tm_main, mbar, 0, h, w, row0, b);
-    if (TileGeom<D>::kHasTail) tma_load_5d(dst + kMainRegionBytes, &p.tm_tail, mbar, 64, h, w,
-                                           row0, b);
-  };
+  // The whole warp runs this loop and waits together; one lane issues.
   auto load_q = [&](int s, const Round& x) -> bool {
     const uint32_t nq = s == 0 ? nq0 : nq1;
     if (!wait_bounded(bar.q_empty(s), (nq & 1u) ^ 1u, abort_flag, p.wait_limit_ns, kSiteLoadQ))
       return false;
-    mbar_arrive_expect_tx(bar.q_full(s), kTile);
-    load_tile(sQ + s * kTile, bar.q_full(s), 0, (2 * x.r + s) * kTileRows, x.b, x.h);
+    if (elect_one()) {
+      const uint32_t dst = sQ + s * G::kQBytes;
+      const int row0 = (2 * x.r + s) * kQRows;
+      mbar_arrive_expect_tx(bar.q_full(s), G::kQBytes);
+      tma_load_5d(dst, &p.tm_q, bar.q_full(s), 0, x.h, 0, row0, x.b);
+      if (G::kHasTail)
+        tma_load_5d(dst + G::kQTail, &p.tm_q_tail, bar.q_full(s), 64, x.h, 0, row0, x.b);
+    }
+    __syncwarp();
     if (s == 0) ++nq0; else ++nq1;
     return true;
+  };
+  auto load_kv = [&](uint32_t dst, uint32_t mbar, int w, int j, const Round& x) {
+    if (elect_one()) {
+      mbar_arrive_expect_tx(mbar, G::kKVBytes);
+      tma_load_5d(dst, &p.tm_kv, mbar, 0, x.h, w, j * G::BK, x.b);
+      if (G::kHasTail)
+        tma_load_5d(dst + G::kKVTail, &p.tm_kv_tail, mbar, 64, x.h, w, j * G::BK, x.b);
+    }
+    __syncwarp();
   };
 
   for (int u = blockIdx.x; ok && u < p.num_units; u += gridDim.x) {
@@ -232,27 +281,22 @@ __device__ void load_role(const AttnParams& p, uint32_t sQ, uint32_t sK, uint32_
       const Round x = make_round(p, u, rr);
       if (!p.reuse || x.first) {
         for (int j = 0; ok && j < nb; ++j) {
-          const int slot = static_cast<int>(kv_ev % R);
-          const uint32_t n = kv_ev / R;
-          if (!wait_bounded(bar.k_empty(slot), (n & 1u) ^ 1u, abort_flag, p.wait_limit_ns,
-                            kSiteLoadK)) {
-            ok = false;
-            break;
-          }
-          if (!wait_bounded(bar.v_empty(slot), (n & 1u) ^ 1u, abort_flag, p.wait_limit_ns,
+          const int slot = pos.slot;
+          if (!wait_bounded(bar.k_empty(slot), pos.phase ^ 1u, abort_flag, p.wait_limit_ns,
+                            kSiteLoadK) ||
+              !wait_bounded(bar.v_empty(slot), pos.phase ^ 1u, abort_flag, p.wait_limit_ns,
                             kSiteLoadV)) {
             ok = false;
             break;
           }
-          mbar_arrive_expect_tx(bar.k_full(slot), kTile);
-          load_tile(sK + slot * kTile, bar.k_full(slot), 1, j * kTileRows, x.b, x.h);
+          load_kv(sK + slot * G::kKVStride, bar.k_full(slot), 1, j, x);
           if (j == 0) {
             // Q tiles right after the first K block so S(0) can start early.
             for (int s = 0; ok && s < x.nslots; ++s) ok = load_q(s, x);
           }
-          mbar_arrive_expect_tx(bar.v_full(slot), kTile);
-          load_tile(sV + slot * kTile, bar.v_full(slot), 2, j * kTileRows, x.b, x.h);
+          load_kv(sV + slot * G::kKVStride, bar.v_full(slot), 2, j, x);
           ++kv_ev;
+          pos.advance(R);
         }
       } else {
         for (int s = 0; ok && s < x.nslots; ++s) ok = load_q(s, x);
@@ -272,63 +316,39 @@ __device__ void load_role(const AttnParams& p, uint32_t sQ, uint32_t sK, uint32_
 }
 
 // ------------------------------------------------------------ MMA issuer
-template <int D>
-__device__ __forceinline__ void issue_scores(uint32_t tmem_s, uint32_t q_addr, uint32_t k_addr,
-                                             int ncols) {
-  const uint32_t idesc = idesc_bf16_m128(static_cast<uint32_t>(ncols), 0u);
-#pragma unroll
-  for (int kk = 0; kk < 4; ++kk) {
-    mma_ss(tmem_s, smem_desc(q_addr + kk * 32, 16, 1024, kSwizzle128),
-           smem_desc(k_addr + kk * 32, 16, 1024, kSwizzle128), idesc, kk > 0 ? 1u : 0u);
-  }
-  if (TileGeom<D>::kHasTail) {
-    mma_ss(tmem_s, smem_desc(q_addr + kMainRegionBytes, 16, 256, kSwizzle32),
-           smem_desc(k_addr + kMainRegionBytes, 16, 256, kSwizzle32), idesc, 1u);
-  }
-}
-
-template <int D>
-__device__ __forceinline__ void issue_values(uint32_t tmem_o, uint32_t tmem_p, uint32_t v_addr,
-                                             int ncols, bool accumulate) {
-  constexpr uint32_t idesc_main = idesc_bf16_m128(64u, 1u);
-  constexpr uint32_t idesc_tail = idesc_bf16_m128(16u, 1u);
-  const int ksteps = ncols / 16;
-  for (int kk = 0; kk < ksteps; ++kk) {
-    const uint32_t acc = (accumulate || kk > 0) ? 1u : 0u;
-    mma_ts(tmem_o, tmem_p + kk * 8,
-           smem_desc(v_addr + kk * 16 * 128, kMainRegionBytes, 1024, kSwizzle128), idesc_main,
-           acc);
-    if (TileGeom<D>::kHasTail) {
-      mma_ts(tmem_o + 64, tmem_p + kk * 8,
-             smem_desc(v_addr + kMainRegionBytes + kk * 16 * 32, kTailRegionBytes, 256,
-                       kSwizzle32),
-             idesc_tail, acc);
-    }
-  }
-}
-
+// Shared-memory descriptors are built once; a K step only moves the start
+// address field (bits [0,14), in 16-byte units), so each step is one add.
 template <int D>
 __device__ void mma_role(const AttnParams& p, uint32_t tmem, uint32_t sQ, uint32_t sK,
                          uint32_t sV, const Barriers& bar, volatile int* abort_flag) {
-  constexpr uint32_t kTile = TileGeom<D>::kBytes;
+  using G = Geom<D>;
   const int R = p.ring;
   const int nb = p.num_kblocks;
-  uint32_t nq0 = 0, nq1 = 0;  // q_full phases consumed per Q slot
-  uint32_t np0 = 0, np1 = 0, np2 = 0;  // p_full phases consumed per channel
-  uint32_t kv_ev = 0;
   const unsigned long long lim = p.wait_limit_ns;
+  uint32_t nq0 = 0, nq1 = 0;  // q_full phases consumed per Q slot
+  uint32_t nf0 = 0, nf1 = 0;  // s_free phases consumed per slot
+  uint32_t np0 = 0, np1 = 0;  // p_full phases consumed per slot
+  RingPos pos{0, 0u};         // ring position of the next unit / round's first K/V event
 
-  auto wait_k = [&](uint32_t ev) -> bool {
-    if (!wait_bounded(bar.k_full(static_cast<int>(ev % R)), (ev / R) & 1u, abort_flag, lim,
-                      kSiteMmaK))
-      return false;
+  const uint64_t q_desc0 = smem_desc(sQ, 16, 1024, kSwizzle128);
+  const uint64_t q_tail0 = smem_desc(sQ + G::kQTail, 16, 256, kSwizzle32);
+  const uint64_t k_desc0 = smem_desc(sK, 16, 1024, kSwizzle128);
+  const uint64_t k_tail0 = smem_desc(sK + G::kKVTail, 16, 256, kSwizzle32);
+  const uint64_t v_desc0 = smem_desc(sV, G::kKVTail, 1024, kSwizzle128);
+  const uint64_t v_tail0 = smem_desc(sV + G::kKVTail, 32 * G::BK, 256, kSwizzle32);
+  constexpr uint64_t kQStep = G::kQBytes >> 4;     // next Q slot
+  constexpr uint64_t kKVStep = G::kKVStride >> 4;  // next ring slot
+  constexpr uint32_t kIdescPV = idesc_bf16_m128(64u, 1u);
+  constexpr uint32_t kIdescPVTail = idesc_bf16_m128(16u, 1u);
+
+  auto wait_k = [&](const RingPos& e) -> bool {
+    if (!wait_bounded(bar.k_full(e.slot), e.phase, abort_flag, lim, kSiteMmaK)) return false;
     tc_fence_after();
     return true;
   };
-  auto wait_v = [&](uint32_t ev) -> bool {
-    if (!wait_bounded(bar.v_full(static_cast<int>(ev % R)), (ev / R) & 1u, abort_flag, lim,
-                      kSiteMmaV))
-      return false;
+  auto wait_v = [&](const RingPos& e) -> bool {
+    if (!wait_bounded(bar.v_full(e.slot), e.phase, abort_flag, lim, kSiteMmaV)) return false;
+    VLA_TRACE_EVENT(kTrMmaV, 0, 0);
     tc_fence_after();
     return true;
   };
@@ -339,94 +359,134 @@ __device__ void mma_role(const AttnParams& p, uint32_t tmem, uint32_t sQ, uint32
     tc_fence_after();
     return true;
   };
-  auto wait_p = [&](int ch) -> bool {
-    const uint32_t np = ch == 0 ? np0 : (ch == 1 ? np1 : np2);
-    if (!wait_bounded(bar.p_full(ch), np & 1u, abort_flag, lim, kSiteMmaP)) return false;
-    if (ch == 0) ++np0; else if (ch == 1) ++np1; else ++np2;
+  auto wait_free = [&](int s) -> bool {
+    const uint32_t nf = s == 0 ? nf0 : nf1;
+    if (!wait_bounded(bar.s_free(s), nf & 1u, abort_flag, lim, kSiteMmaFree)) return false;
+    VLA_TRACE_EVENT(kTrMmaFree, s, 0);
+    if (s == 0) ++nf0; else ++nf1;
     tc_fence_after();
     return true;
   };
-  // S into buffer `buf` for Q slot `s` and key block j (event ev), signalled
-  // on channel `ch`.
-  auto scores = [&](int s, int buf, int ch, int j, uint32_t ev) {
-    VLA_TRACE_EVENT(kTrMmaS, s, j);
-    issue_scores<D>(tmem + buf * 256, sQ + s * kTile, sK + static_cast<int>(ev % R) * kTile,
-                    block_cols(p.N, j));
-    mma_commit(bar.s_full(ch));
+  auto wait_p = [&](int s) -> bool {
+    const uint32_t np = s == 0 ? np0 : np1;
+    if (!wait_bounded(bar.p_full(s), np & 1u, abort_flag, lim, kSiteMmaP)) return false;
+    VLA_TRACE_EVENT(kTrMmaP, s, 0);
+    if (s == 0) ++np0; else ++np1;
+    tc_fence_after();
+    return true;
   };
-  auto values = [&](int s, int buf, int j, uint32_t ev) {
+  // The whole warp runs the issue loop and waits together; one lane issues
+  // the tensor-core instructions and commits.
+  auto commit = [&](uint32_t mbar) {
+    if (elect_one()) mma_commit(mbar);
+    __syncwarp();
+  };
+  // S of Q slot s against key block j held in ring slot `kslot`.
+  auto scores = [&](int s, int j, int kslot) {
+    VLA_TRACE_EVENT(kTrMmaS, s, j);
+    const uint32_t idesc = idesc_bf16_m128(static_cast<uint32_t>(block_cols<G::BK>(p.N, j)), 0u);
+    const uint32_t d_tmem = tmem + s * 256;
+    const uint64_t qd = q_desc0 + s * kQStep;
+    const uint64_t kd = k_desc0 + kslot * kKVStep;
+    if (elect_one()) {
+#pragma unroll
+      for (int kk = 0; kk < 4; ++kk)
+        mma_ss(d_tmem, qd + 2 * kk, kd + 2 * kk, idesc, kk > 0 ? 1u : 0u);  // 16 ch = 32 B
+      if (G::kHasTail)
+        mma_ss(d_tmem, q_tail0 + s * kQStep, k_tail0 + kslot * kKVStep, idesc, 1u);
+      mma_commit(bar.s_full(s));
+    }
+    __syncwarp();
+    VLA_TRACE_EVENT(kTrMmaSDone, s, j);
+  };
+  // O_s (+)= P_s V_j, V_j in ring slot `vslot`.
+  auto values = [&](int s, int j, int vslot) {
     VLA_TRACE_EVENT(kTrMmaPV, s, j);
-    issue_values<D>(tmem + s * 256 + 128, tmem + buf * 256, sV + static_cast<int>(ev % R) * kTile,
-                    block_cols(p.N, j), j > 0);
-    mma_commit(bar.o_prog(s));
+    const int ksteps = block_cols<G::BK>(p.N, j) / 16;
+    const uint32_t o_tmem = tmem + s * 256 + G::kColO;
+    const uint32_t p_tmem = tmem + s * 256 + G::kColP;
+    const uint64_t vd = v_desc0 + vslot * kKVStep;
+    const uint64_t vt = v_tail0 + vslot * kKVStep;
+    if (elect_one()) {
+      for (int kk = 0; kk < ksteps; ++kk) {
+        const uint32_t acc = (j > 0 || kk > 0) ? 1u : 0u;
+        mma_ts(o_tmem, p_tmem + kk * 8, vd + kk * 128, kIdescPV, acc);  // 16 keys x 128 B
+        if (G::kHasTail) mma_ts(o_tmem + 64, p_tmem + kk * 8, vt + kk * 32, kIdescPVTail, acc);
+      }
+      mma_commit(bar.o_prog(s));
+    }
+    __syncwarp();
+    VLA_TRACE_EVENT(kTrMmaPVDone, s, j);
   };
 
   bool ok = true;
   for (int u = blockIdx.x; ok && u < p.num_units; u += gridDim.x) {
-    const uint32_t unit_ev0 = kv_ev;
+    const RingPos unit_pos = pos;
     for (int rr = 0; ok && rr < p.rounds_per_unit; ++rr) {
       const Round x = make_round(p, u, rr);
-      const uint32_t ev0 = p.reuse ? unit_ev0 : kv_ev;
+      const int ns = x.nslots;
       const bool release = !p.reuse || x.last;
-      if (x.nslots == 2) {
-        if (!(ok = wait_k(ev0))) break;
-        for (int s = 0; s < 2; ++s) {
-          if (!(ok = wait_q(s))) break;
-          scores(s, s, s, 0, ev0);
-          if (nb == 1) mma_commit(bar.q_empty(s));
+      RingPos cur = p.reuse ? unit_pos : pos;  // event of key block j
+      RingPos k2 = cur;                         // event of the next S to issue
+      // S of the first key block for every slot (the previous round's last S
+      // of each slot was read out before its s_free phase was consumed).
+      if (!(ok = wait_k(k2))) break;
+      for (int s = 0; ok && s < ns; ++s) {
+        if (!(ok = wait_q(s))) break;
+        scores(s, 0, k2.slot);
+        if (nb == 1) commit(bar.q_empty(s));
+      }
+      if (!ok) break;
+      if (release) commit(bar.k_empty(k2.slot));
+      k2.advance(R);
+      // S of the second key block once each slot has read its first S.
+      if (nb > 1) {
+        if (!(ok = wait_k(k2))) break;
+        for (int s = 0; ok && s < ns; ++s) {
+          if (!(ok = wait_free(s))) break;
+          scores(s, 1, k2.slot);
+          if (nb == 2) commit(bar.q_empty(s));
         }
         if (!ok) break;
-        if (release) mma_commit(bar.k_empty(static_cast<int>(ev0 % R)));
-        for (int j = 0; ok && j < nb; ++j) {
-          const uint32_t ev = ev0 + j;
-          if (!(ok = wait_v(ev))) break;
-          for (int s = 0; s < 2; ++s) {
-            if (!(ok = wait_p(s))) break;
-            values(s, s, j, ev);
-            if (j + 1 < nb) {
-              if (s == 0 && !(ok = wait_k(ev + 1))) break;
-              scores(s, s, s, j + 1, ev + 1);
-              if (j + 1 == nb - 1) mma_commit(bar.q_empty(s));
+        if (release) commit(bar.k_empty(k2.slot));
+        k2.advance(R);
+      }
+      // Steady state, in the order the softmax warpgroups produce events:
+      // P_s(j) -> P V; slot s then reads S_s(j+1) -> S_s(j+2) into its buffer.
+      for (int j = 0; ok && j < nb; ++j) {
+        if (!(ok = wait_v(cur))) break;
+        const bool next_s = j + 2 < nb;
+        if (next_s && !(ok = wait_k(k2))) break;
+        for (int s = 0; s < ns; ++s) {
+          if (!(ok = wait_p(s))) break;
+          values(s, j, cur.slot);
+          if (j + 1 < nb) {
+            if (!(ok = wait_free(s))) break;
+            if (next_s) {
+              scores(s, j + 2, k2.slot);
+              if (j + 2 == nb - 1) commit(bar.q_empty(s));
             }
           }
-          if (!ok) break;
-          if (release) {
-            mma_commit(bar.v_empty(static_cast<int>(ev % R)));
-            if (j + 1 < nb) mma_commit(bar.k_empty(static_cast<int>((ev + 1) % R)));
-          }
         }
-      } else {
-        // Half round: slot 0 alone, S alternating between buffers 0 and 1
-        // (channels 0 and 2).
-        if (!(ok = wait_q(0))) break;
-        for (int j = 0; j < 2 && j < nb; ++j) {
-          if (!(ok = wait_k(ev0 + j))) break;
-          scores(0, j, 2 * j, j, ev0 + j);
-          if (j == nb - 1) mma_commit(bar.q_empty(0));
-          if (release) mma_commit(bar.k_empty(static_cast<int>((ev0 + j) % R)));
+        if (!ok) break;
+        if (release) {
+          commit(bar.v_empty(cur.slot));
+          if (next_s) commit(bar.k_empty(k2.slot));
         }
-        for (int j = 0; ok && j < nb; ++j) {
-          const uint32_t ev = ev0 + j;
-          const int buf = j & 1;
-          if (!(ok = wait_v(ev))) break;
-          if (!(ok = wait_p(2 * buf))) break;
-          values(0, buf, j, ev);
-          if (release) mma_commit(bar.v_empty(static_cast<int>(ev % R)));
-          if (j + 2 < nb) {
-            if (!(ok = wait_k(ev + 2))) break;
-            scores(0, buf, 2 * buf, j + 2, ev + 2);
-            if (j + 2 == nb - 1) mma_commit(bar.q_empty(0));
-            if (release) mma_commit(bar.k_empty(static_cast<int>((ev + 2) % R)));
-          }
-        }
+        if (next_s) k2.advance(R);
+        cur.advance(R);
       }
-      if (!p.reuse) kv_ev += nb;
+      if (!ok) break;
+      if (nb == 1) {
+        for (int s = 0; ok && s < ns; ++s) ok = wait_free(s);
+        if (!ok) break;
+      }
+      pos = cur;  // first event after this round (reuse: after the unit)
     }
-    if (p.reuse) kv_ev += nb;
   }
   // Every tensor-core operation issued above must finish before the tensor
   // memory is freed.
-  mma_commit(bar.drain());
+  commit(bar.drain());
   wait_drain(bar.drain(), 0u, kDrainLimitNs);
 }
 
@@ -436,23 +496,29 @@ struct SoftState {
   float l_run;  // running sum of weights
 };
 
-// One key block for one query row: S (fp32, NC valid columns at compile time,
-// nvalid at run time) -> running max / sum, P (bf16 pairs) into the S buffer,
-// O rescaled when the maximum grows.  Returns false on abort.
+// One key block for one query row.  Reads S (NC columns at compile time,
+// nvalid valid at run time), signals that S has been read, updates the
+// running max / sum, stores P, rescales O when the maximum grew.  Returns
+// false on abort.
 template <int D, int NC>
 __device__ __forceinline__ bool softmax_block(const AttnParams& p, SoftState& st, uint32_t tS,
-                                              uint32_t tO, int nvalid, bool first_block,
-                                              bool use_token, uint32_t tok_wait_bar,
-                                              uint32_t tok_wait_parity, uint32_t tok_arrive_bar,
-                                              uint32_t o_prog_bar, uint32_t o_prog_parity,
+                                              uint32_t tO, uint32_t tP, int nvalid, int j,
+                                              bool use_token, const Barriers& bar, int s,
+                                              uint32_t tok_parity, uint32_t o_parity,
                                               volatile int* abort_flag, int lane) {
-  constexpr int DP = TileGeom<D>::kHasTail ? 80 : 64;
+  using G = Geom<D>;
   const float c = p.c;
-  uint32_t sr[128];
-  tmem_ld128(tS, sr);
   float x[NC];
+  {
+    uint32_t sr[128];
+    tmem_ld128(tS, sr);
 #pragma unroll
-  for (int i = 0; i < NC; ++i) x[i] = __uint_as_float(sr[i]);
+    for (int i = 0; i < NC; ++i) x[i] = __uint_as_float(sr[i]);
+  }
+  // S is in registers: the tensor core may overwrite it with the next block.
+  tc_fence_before();
+  __syncwarp();
+  if (lane == 0) mbar_arrive(bar.s_free(s));
   if (nvalid < NC) {
 #pragma unroll
     for (int i = 0; i < NC; ++i)
@@ -486,12 +552,12 @@ __device__ __forceinline__ bool softmax_block(const AttnParams& p, SoftState& st
     st.l_run *= alpha;
   }
   const float mc = st.m_run * c;
-  VLA_TRACE_EVENT(kTrSoftMax, 0, 0);
+  VLA_TRACE_EVENT(kTrSoftMax, s, j);
   if (use_token) {
-    if (!wait_bounded(tok_wait_bar, tok_wait_parity, abort_flag, p.wait_limit_ns, kSiteSoftTok))
+    if (!wait_bounded(bar.tok(s), tok_parity, abort_flag, p.wait_limit_ns, kSiteSoftTok))
       return false;
   }
-  VLA_TRACE_EVENT(kTrSoftTok, 0, 0);
+  VLA_TRACE_EVENT(kTrSoftTok, s, j);
   float lsum[4] = {0.f, 0.f, 0.f, 0.f};
   uint32_t pk[64];
 #pragma unroll
@@ -503,32 +569,32 @@ __device__ __forceinline__ bool softmax_block(const AttnParams& p, SoftState& st
   }
 #pragma unroll
   for (int i = NC / 2; i < 64; ++i) pk[i] = 0u;
-  VLA_TRACE_EVENT(kTrSoftExp, 0, 0);
   if (use_token) {
     __syncwarp();
-    if (lane == 0) mbar_arrive(tok_arrive_bar);
+    if (lane == 0) mbar_arrive(bar.tok(1 - s));
   }
+  VLA_TRACE_EVENT(kTrSoftExp, s, j);
   st.l_run += (lsum[0] + lsum[1]) + (lsum[2] + lsum[3]);
-  tmem_st64(tS, pk);
-  if (!first_block) {
-    // P V of the previous block has to be complete before O is touched (and
-    // this observes every phase of the O progress barrier in order).
-    if (!wait_bounded(o_prog_bar, o_prog_parity, abort_flag, p.wait_limit_ns, kSiteSoftO))
+  if (j > 0) {
+    // P V of the previous block must be done before P is overwritten and
+    // before O is touched (this observes every phase of o_prog in order).
+    if (!wait_bounded(bar.o_prog(s), o_parity, abort_flag, p.wait_limit_ns, kSiteSoftO))
       return false;
     tc_fence_after();
-    if (rescale) {
-      uint32_t ob[64];
-      tmem_ld64(tO, ob);
+  }
+  tmem_st64(tP, pk);
+  if (j > 0 && rescale) {
+    uint32_t ob[64];
+    tmem_ld64(tO, ob);
 #pragma unroll
-      for (int i = 0; i < 64; ++i) ob[i] = __float_as_uint(__uint_as_float(ob[i]) * alpha);
-      tmem_st64(tO, ob);
-      if (DP > 64) {
-        uint32_t ot[16];
-        tmem_ld16(tO + 64, ot);
+    for (int i = 0; i < 64; ++i) ob[i] = __float_as_uint(__uint_as_float(ob[i]) * alpha);
+    tmem_st64(tO, ob);
+    if (G::DP > 64) {
+      uint32_t ot[16];
+      tmem_ld16(tO + 64, ot);
 #pragma unroll
-        for (int i = 0; i < 16; ++i) ot[i] = __float_as_uint(__uint_as_float(ot[i]) * alpha);
-        tmem_st16(tO + 64, ot);
-      }
+      for (int i = 0; i < 16; ++i) ot[i] = __float_as_uint(__uint_as_float(ot[i]) * alpha);
+      tmem_st16(tO + 64, ot);
     }
   }
   tmem_wait_st();
@@ -536,15 +602,17 @@ __device__ __forceinline__ bool softmax_block(const AttnParams& p, SoftState& st
 }
 
 template <int D>
-__device__ __forceinline__ bool softmax_block_dispatch(
-    const AttnParams& p, SoftState& st, uint32_t tS, uint32_t tO, int ncols, int nvalid,
-    bool first_block, bool use_token, uint32_t tw, uint32_t twp, uint32_t ta, uint32_t ob,
-    uint32_t obp, volatile int* abort_flag, int lane) {
-#define VLA_SB(NC)                                                                          \
-  return softmax_block<D, NC>(p, st, tS, tO, nvalid, first_block, use_token, tw, twp, ta, ob, \
-                              obp, abort_flag, lane)
+__device__ __forceinline__ bool softmax_block_dispatch(const AttnParams& p, SoftState& st,
+                                                       uint32_t tS, uint32_t tO, uint32_t tP,
+                                                       int ncols, int nvalid, int j,
+                                                       bool use_token, const Barriers& bar,
+                                                       int s, uint32_t tp, uint32_t op,
+                                                       volatile int* abort_flag, int lane) {
+#define VLA_SB(NC)                                                                       \
+  return softmax_block<D, NC>(p, st, tS, tO, tP, nvalid, j, use_token, bar, s, tp, op, \
+                              abort_flag, lane)
+  if (ncols >= Geom<D>::BK) VLA_SB(Geom<D>::BK);
   switch (ncols) {
-    case 128: VLA_SB(128);
     case 112: VLA_SB(112);
     case 96: VLA_SB(96);
     case 80: VLA_SB(80);
@@ -559,16 +627,18 @@ __device__ __forceinline__ bool softmax_block_dispatch(
 template <int D>
 __device__ void softmax_role(const AttnParams& p, uint32_t tmem, const Barriers& bar,
                              volatile int* abort_flag, int warp, int lane) {
-  constexpr int DP = TileGeom<D>::kHasTail ? 80 : 64;
+  using G = Geom<D>;
   const int s = warp >> 2;  // Q slot of this warpgroup
   const int quad = warp & 3;
   const int row_in_tile = quad * 32 + lane;
   const uint32_t lane_bits = static_cast<uint32_t>(quad * 32) << 16;
-  const uint32_t tO = tmem + lane_bits + s * 256 + 128;
+  const uint32_t tS = tmem + lane_bits + s * 256;
+  const uint32_t tO = tS + G::kColO;
+  const uint32_t tP = tS + G::kColP;
   const int nb = p.num_kblocks;
-  uint32_t ns0 = 0, ns1 = 0, ns2 = 0;  // s_full phases consumed per channel
-  uint32_t npv = 0;           // completions of o_prog[s] accounted for
-  uint32_t ntok = 0;          // exp2 turns taken by this warpgroup
+  uint32_t ns = 0;    // s_full phases consumed
+  uint32_t npv = 0;   // o_prog phases consumed
+  uint32_t ntok = 0;  // exp2 turns taken
 
   for (int u = blockIdx.x; u < p.num_units; u += gridDim.x) {
     for (int rr = 0; rr < p.rounds_per_unit; ++rr) {
@@ -578,26 +648,21 @@ __device__ void softmax_role(const AttnParams& p, uint32_t tmem, const Barriers&
       const int tile = 2 * x.r + s;
       SoftState st{-INFINITY, 0.0f};
       for (int j = 0; j < nb; ++j) {
-        const int buf = full ? s : (j & 1);
-        const int ch = full ? s : 2 * buf;
-        const uint32_t ns = ch == 0 ? ns0 : (ch == 1 ? ns1 : ns2);
-        if (!wait_bounded(bar.s_full(ch), ns & 1u, abort_flag, p.wait_limit_ns, kSiteSoftS))
+        if (!wait_bounded(bar.s_full(s), ns & 1u, abort_flag, p.wait_limit_ns, kSiteSoftS))
           return;
-        if (ch == 0) ++ns0; else if (ch == 1) ++ns1; else ++ns2;
-        VLA_TRACE_EVENT(kTrSoftS, s, j);
+        ++ns;
         tc_fence_after();
-        const uint32_t tS = tmem + lane_bits + buf * 256;
-        // Slot 0 takes exp2 turns 0, 1, 2, ... after slot 1's turns -1, 0, 1, ...
-        const uint32_t tw = bar.tok(s);
-        const uint32_t twp = s == 0 ? ((ntok & 1u) ^ 1u) : (ntok & 1u);
+        VLA_TRACE_EVENT(kTrSoftS, s, j);
+        // Slot 0 takes exp2 turns 0, 1, 2, ... right after slot 1's turns -1, 0, 1, ...
+        const uint32_t tp = s == 0 ? ((ntok & 1u) ^ 1u) : (ntok & 1u);
         const bool ok = softmax_block_dispatch<D>(
-            p, st, tS, tO, block_cols(p.N, j), min(kTileRows, p.N - j * kTileRows), j == 0, full,
-            tw, twp, bar.tok(1 - s), bar.o_prog(s), (npv + j - 1) & 1u, abort_flag, lane);
+            p, st, tS, tO, tP, block_cols<G::BK>(p.N, j), min(G::BK, p.N - j * G::BK), j, full,
+            bar, s, tp, (npv + j - 1) & 1u, abort_flag, lane);
         if (!ok) return;
         if (full) ++ntok;
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(bar.p_full(ch));
+        if (lane == 0) mbar_arrive(bar.p_full(s));
         VLA_TRACE_EVENT(kTrSoftP, s, j);
       }
       // Epilogue: wait for the last P V, then O / l -> bf16, 16-byte stores.
@@ -611,8 +676,8 @@ __device__ void softmax_role(const AttnParams& p, uint32_t tmem, const Barriers&
       uint32_t ob[64];
       tmem_ld64(tO, ob);
       uint32_t ot[16];
-      if (DP > 64) tmem_ld16(tO + 64, ot);
-      const int row = tile * kTileRows + row_in_tile;
+      if (G::DP > 64) tmem_ld16(tO + 64, ot);
+      const int row = tile * kQRows + row_in_tile;
       if (row < p.N) {
         uint4* dst = reinterpret_cast<uint4*>(
             p.o + ((static_cast<size_t>(x.b) * p.N + row) * p.H + x.h) * D);
@@ -639,14 +704,14 @@ __device__ void softmax_role(const AttnParams& p, uint32_t tmem, const Barriers&
 // ------------------------------------------------------------ kernel
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_constant__ AttnParams p) {
+  using G = Geom<D>;
   extern __shared__ uint8_t smem_raw[];
-  constexpr uint32_t kTile = TileGeom<D>::kBytes;
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
   const uint32_t sQ = base;
-  const uint32_t sK = sQ + 2 * kTile;
-  const uint32_t sV = sK + p.ring * kTile;
-  const uint32_t sBar = sV + p.ring * kTile;
+  const uint32_t sK = sQ + 2 * G::kQBytes;
+  const uint32_t sV = sK + p.ring * G::kKVStride;
+  const uint32_t sBar = sV + p.ring * G::kKVStride;
   uint8_t* bar_generic = smem_raw + (sBar - raw);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_generic + 8 * kNumBarriers);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(bar_generic + 8 * kNumBarriers + 4);
@@ -659,12 +724,11 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
     for (int s = 0; s < 2; ++s) {
       mbar_init(bar.q_full(s), 1);
       mbar_init(bar.q_empty(s), 1);
+      mbar_init(bar.s_full(s), 1);
+      mbar_init(bar.s_free(s), 4);
+      mbar_init(bar.p_full(s), 4);
       mbar_init(bar.o_prog(s), 1);
       mbar_init(bar.tok(s), 4);
-    }
-    for (int ch = 0; ch < 3; ++ch) {
-      mbar_init(bar.s_full(ch), 1);
-      mbar_init(bar.p_full(ch), 4);
     }
     for (int i = 0; i < kMaxRing; ++i) {
       mbar_init(bar.k_full(i), 1);
@@ -678,8 +742,12 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
   }
   VLA_TRACE_INIT();
   if (warp == kLoadWarp && lane == 0) {
-    prefetch_tmap(&p.tm_main);
-    if (TileGeom<D>::kHasTail) prefetch_tmap(&p.tm_tail);
+    prefetch_tmap(&p.tm_q);
+    prefetch_tmap(&p.tm_kv);
+    if (G::kHasTail) {
+      prefetch_tmap(&p.tm_q_tail);
+      prefetch_tmap(&p.tm_kv_tail);
+    }
   }
   if (warp == kMmaWarp) {
     tmem_alloc(smem_u32(tmem_slot), kTmemCols);
@@ -691,10 +759,10 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
   const uint32_t tmem = *tmem_slot;
 
   if (warp == kLoadWarp) {
-    if (lane == 0) load_role<D>(p, sQ, sK, sV, bar, abort_flag);
+    load_role<D>(p, sQ, sK, sV, bar, abort_flag);
     __syncwarp();
   } else if (warp == kMmaWarp) {
-    if (lane == 0) mma_role<D>(p, tmem, sQ, sK, sV, bar, abort_flag);
+    mma_role<D>(p, tmem, sQ, sK, sV, bar, abort_flag);
     __syncwarp();
   } else if (warp < 8) {
     softmax_role<D>(p, tmem, bar, abort_flag, warp, lane);

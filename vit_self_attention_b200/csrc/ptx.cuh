@@ -246,6 +246,18 @@ __host__ __device__ constexpr uint32_t idesc_bf16_m128(uint32_t n, uint32_t b_mn
          ((128u >> 4) << 24);
 }
 
+// ------------------------------------------------------------------- warp
+// True in exactly one lane of the (converged) warp.
+__device__ __forceinline__ bool elect_one() {
+  uint32_t pred;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "elect.sync _|p, 0xffffffff;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(pred));
+  return pred != 0;
+}
+
 // ------------------------------------------------------------------- math
 __device__ __forceinline__ float ex2_approx(float x) {
   float y;

@@ -133,14 +133,14 @@ int check_device_range(const DriverFns& fns, const void* p, size_t bytes, int de
 }
 
 int encode_map(const DriverFns& fns, CUtensorMap* map, const void* qkv, int B, int N, int H,
-               int d, uint32_t box_c, CUtensorMapSwizzle swizzle) {
+               int d, uint32_t box_c, uint32_t box_rows, CUtensorMapSwizzle swizzle) {
   const cuuint64_t dims[5] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(H), 3u,
                               static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(B)};
   const cuuint64_t tok = 3ull * H * d * 2ull;
   const cuuint64_t strides[4] = {static_cast<cuuint64_t>(d) * 2ull,
                                  static_cast<cuuint64_t>(H) * d * 2ull, tok,
                                  tok * static_cast<cuuint64_t>(N)};
-  const cuuint32_t box[5] = {box_c, 1u, 1u, static_cast<cuuint32_t>(vla::kTileRows), 1u};
+  const cuuint32_t box[5] = {box_c, 1u, 1u, box_rows, 1u};
   const cuuint32_t elem_strides[5] = {1u, 1u, 1u, 1u, 1u};
   const CUresult rc = fns.encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void*>(qkv),
                                  dims, strides, box, elem_strides, CU_TENSOR_MAP_INTERLEAVE_NONE,
@@ -171,19 +171,26 @@ int check_args(const void* q, const void* k, const void* v, const void* o, int B
 template <int D>
 int launch(const void* q, void* o, int B, int N, int H, float scale, cudaStream_t stream,
            const DeviceInfo& di, int dev, const DriverFns& fns) {
-  constexpr uint32_t kTile = vla::TileGeom<D>::kBytes;
+  using G = vla::Geom<D>;
   vla::AttnParams prm;
   std::memset(&prm, 0, sizeof(prm));
-  int rc = encode_map(fns, &prm.tm_main, q, B, N, H, D, 64u, CU_TENSOR_MAP_SWIZZLE_128B);
+  int rc = encode_map(fns, &prm.tm_q, q, B, N, H, D, 64u, vla::kQRows, CU_TENSOR_MAP_SWIZZLE_128B);
   if (rc != VLA_ATTN_OK) return rc;
-  if (D > 64) {
-    rc = encode_map(fns, &prm.tm_tail, q, B, N, H, D, 16u, CU_TENSOR_MAP_SWIZZLE_32B);
+  rc = encode_map(fns, &prm.tm_kv, q, B, N, H, D, 64u, G::BK, CU_TENSOR_MAP_SWIZZLE_128B);
+  if (rc != VLA_ATTN_OK) return rc;
+  if (G::kHasTail) {
+    rc = encode_map(fns, &prm.tm_q_tail, q, B, N, H, D, 16u, vla::kQRows,
+                    CU_TENSOR_MAP_SWIZZLE_32B);
+    if (rc != VLA_ATTN_OK) return rc;
+    rc = encode_map(fns, &prm.tm_kv_tail, q, B, N, H, D, 16u, G::BK, CU_TENSOR_MAP_SWIZZLE_32B);
     if (rc != VLA_ATTN_OK) return rc;
   }
-  const int nb = (N + vla::kTileRows - 1) / vla::kTileRows;
+  const int nb = (N + G::BK - 1) / G::BK;
+  const int nq = (N + vla::kQRows - 1) / vla::kQRows;
   const int max_smem = di.max_smem_optin - static_smem_bytes<D>();
-  int ring = (max_smem - static_cast<int>(2 * kTile + vla::kBarrierRegionBytes + vla::kAlignSlack)) /
-             static_cast<int>(2 * kTile);
+  int ring = (max_smem - static_cast<int>(2 * G::kQBytes + vla::kBarrierRegionBytes +
+                                          vla::kAlignSlack)) /
+             static_cast<int>(2 * G::kKVStride);
   if (ring > vla::kMaxRing) ring = vla::kMaxRing;
   if (ring < 2) return VLA_ATTN_ERR_DEVICE;
   const uint32_t smem = vla::smem_bytes_for_ring<D>(ring);
@@ -193,8 +200,8 @@ int launch(const void* q, void* o, int B, int N, int H, float scale, cudaStream_
   prm.N = N;
   prm.H = H;
   prm.num_kblocks = nb;
-  prm.num_qtiles = nb;
-  prm.rounds_per_head = (nb + 1) / 2;
+  prm.num_qtiles = nq;
+  prm.rounds_per_head = (nq + 1) / 2;
   const long long heads = static_cast<long long>(B) * H;
   prm.rounds_per_unit = heads >= di.sm_count ? prm.rounds_per_head : 1;
   prm.units_per_head = prm.rounds_per_head / prm.rounds_per_unit;
