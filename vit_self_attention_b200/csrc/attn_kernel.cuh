@@ -9,21 +9,21 @@
 // goes to memory; section 3.2: the qkv linear feeds the attention module).
 //
 // Blackwell mapping (one persistent CTA per SM, 384 threads = 3 warpgroups):
-//   warp 9      TMA producer: Q tiles (128 query rows) into two Q slots, K and
+//   warp 1      TMA producer: Q tiles (128 query rows) into two Q slots, K and
 //               V blocks (BK keys) into a ring of `ring` slots.  With `reuse`,
 //               a head's K/V blocks are loaded once and serve all of that
 //               head's Q tiles.
-//   warp 8      tcgen05 issuer (one thread): S = Q K^T into tensor memory
-//               (SS MMA, M=128, N=keys of the block, K=16 steps over d) and
-//               O += P V with P read from tensor memory (TS MMA, N=64, plus
-//               N=16 for d=72).
-//   warps 0-7   softmax, one warpgroup per Q slot, one thread per query row
+//   warp 0      tcgen05 issuer of S = Q K^T into tensor memory (SS MMA, M=128,
+//               N=keys of the block, K=16 steps over d).
+//   warp 2      tcgen05 issuer of O += P V with P read from tensor memory (TS
+//               MMA, N=64, plus N=16 for d=72).
+//   warps 4-11  softmax, one warpgroup per Q slot, one thread per query row
 //               (= tensor-memory lane): online softmax in fp32 with exp2 and a
 //               pre-scaled log2(e), P as bf16 pairs in its own tensor-memory
 //               columns, O rescaled in tensor memory only when the running
 //               maximum grows by more than 2^8, epilogue O / l -> bf16 with
 //               16-byte stores.
-//   warps 10-11 idle.
+//   warp 3      idle.
 //
 // Pipelining.  A softmax thread signals "S consumed" as soon as it has the S
 // row of block j in registers, so the tensor core computes S of block j+1
@@ -61,12 +61,14 @@
 namespace vla {
 
 constexpr int kQRows = 128;  // query rows per tile = TMEM lanes = MMA M
-constexpr int kMmaWarp = 8;
-constexpr int kLoadWarp = 9;
+constexpr int kMmaWarp = 0;    // S = Q K^T issuer; also allocates tensor memory
+constexpr int kLoadWarp = 1;   // TMA producer
+constexpr int kPvWarp = 2;     // O += P V issuer
+constexpr int kSoftmaxWarp0 = 4;
 constexpr int kThreads = 384;
 constexpr int kMaxRing = 6;
 constexpr uint32_t kTmemCols = 512;
-constexpr int kNumBarriers = 14 + 4 * kMaxRing + 1;
+constexpr int kNumBarriers = 14 + 4 * kMaxRing + 2;
 constexpr uint32_t kBarrierRegionBytes = 512;  // barriers + tmem address + abort flag
 constexpr uint32_t kAlignSlack = 1024;
 constexpr unsigned long long kDrainLimitNs = 100000000ull;
@@ -95,6 +97,9 @@ enum : int {
 #endif
 #ifndef VLA_TRACE_INIT
 #define VLA_TRACE_INIT() ((void)0)
+#endif
+#ifndef VLA_TRACE_END
+#define VLA_TRACE_END() ((void)0)
 #endif
 
 template <int D>
@@ -155,7 +160,7 @@ struct Barriers {
   __device__ uint32_t k_empty(int i) const { return base + 8u * (14 + kMaxRing + i); }
   __device__ uint32_t v_full(int i) const { return base + 8u * (14 + 2 * kMaxRing + i); }
   __device__ uint32_t v_empty(int i) const { return base + 8u * (14 + 3 * kMaxRing + i); }
-  __device__ uint32_t drain() const { return base + 8u * (14 + 4 * kMaxRing); }
+  __device__ uint32_t drain(int i) const { return base + 8u * (14 + 4 * kMaxRing + i); }
 };
 
 // Bounded wait for the phase of `bar` with the given parity, executed by a
@@ -315,12 +320,18 @@ __device__ void load_role(const AttnParams& p, uint32_t sQ, uint32_t sK, uint32_
   }
 }
 
-// ------------------------------------------------------------ MMA issuer
+// ------------------------------------------------------------ MMA issuers
+// Two warps issue tensor-core work: the score warp issues S = Q K^T (waiting
+// for each slot to have read its previous S), the value warp issues
+// O += P V (waiting for each slot's P).  Issue blocks the issuing thread for
+// about the duration of the MMA, so separate issuers keep each chain
+// responsive.  They touch disjoint tensor-memory columns (S vs P / O).
 // Shared-memory descriptors are built once; a K step only moves the start
 // address field (bits [0,14), in 16-byte units), so each step is one add.
 template <int D>
 __device__ void mma_role(const AttnParams& p, uint32_t tmem, uint32_t sQ, uint32_t sK,
-                         uint32_t sV, const Barriers& bar, volatile int* abort_flag) {
+                         uint32_t sV, const Barriers& bar, volatile int* abort_flag,
+                         bool score_warp) {
   using G = Geom<D>;
   const int R = p.ring;
   const int nb = p.num_kblocks;
@@ -426,68 +437,56 @@ __device__ void mma_role(const AttnParams& p, uint32_t tmem, uint32_t sQ, uint32
       const Round x = make_round(p, u, rr);
       const int ns = x.nslots;
       const bool release = !p.reuse || x.last;
-      RingPos cur = p.reuse ? unit_pos : pos;  // event of key block j
-      RingPos k2 = cur;                         // event of the next S to issue
-      // S of the first key block for every slot (the previous round's last S
-      // of each slot was read out before its s_free phase was consumed).
-      if (!(ok = wait_k(k2))) break;
-      for (int s = 0; ok && s < ns; ++s) {
-        if (!(ok = wait_q(s))) break;
-        scores(s, 0, k2.slot);
-        if (nb == 1) commit(bar.q_empty(s));
-      }
-      if (!ok) break;
-      if (release) commit(bar.k_empty(k2.slot));
-      k2.advance(R);
-      // S of the second key block once each slot has read its first S.
-      if (nb > 1) {
-        if (!(ok = wait_k(k2))) break;
+      RingPos cur = p.reuse ? unit_pos : pos;  // K/V event of key block j
+      if (score_warp) {
+        // S of the first key block for every slot (the previous round's last
+        // S of each slot was read out before its s_free phase was consumed).
+        if (!(ok = wait_k(cur))) break;
         for (int s = 0; ok && s < ns; ++s) {
-          if (!(ok = wait_free(s))) break;
-          scores(s, 1, k2.slot);
-          if (nb == 2) commit(bar.q_empty(s));
+          if (!(ok = wait_q(s))) break;
+          scores(s, 0, cur.slot);
+          if (nb == 1) commit(bar.q_empty(s));
         }
         if (!ok) break;
-        if (release) commit(bar.k_empty(k2.slot));
-        k2.advance(R);
-      }
-      // Steady state, in the order the softmax warpgroups produce events:
-      // P_s(j) -> P V; slot s then reads S_s(j+1) -> S_s(j+2) into its buffer.
-      for (int j = 0; ok && j < nb; ++j) {
-        if (!(ok = wait_v(cur))) break;
-        const bool next_s = j + 2 < nb;
-        if (next_s && !(ok = wait_k(k2))) break;
-        for (int s = 0; s < ns; ++s) {
-          if (!(ok = wait_p(s))) break;
-          values(s, j, cur.slot);
-          if (j + 1 < nb) {
+        if (release) commit(bar.k_empty(cur.slot));
+        // S of block j+1 for slot s as soon as slot s has read S of block j.
+        for (int j = 0; ok && j + 1 < nb; ++j) {
+          cur.advance(R);
+          if (!(ok = wait_k(cur))) break;
+          for (int s = 0; s < ns; ++s) {
             if (!(ok = wait_free(s))) break;
-            if (next_s) {
-              scores(s, j + 2, k2.slot);
-              if (j + 2 == nb - 1) commit(bar.q_empty(s));
-            }
+            scores(s, j + 1, cur.slot);
+            if (j + 1 == nb - 1) commit(bar.q_empty(s));
           }
+          if (!ok) break;
+          if (release) commit(bar.k_empty(cur.slot));
         }
         if (!ok) break;
-        if (release) {
-          commit(bar.v_empty(cur.slot));
-          if (next_s) commit(bar.k_empty(k2.slot));
-        }
-        if (next_s) k2.advance(R);
+        for (int s = 0; ok && s < ns; ++s) ok = wait_free(s);  // last block read out
+        if (!ok) break;
         cur.advance(R);
-      }
-      if (!ok) break;
-      if (nb == 1) {
-        for (int s = 0; ok && s < ns; ++s) ok = wait_free(s);
+      } else {
+        // P V of block j for slot s as soon as slot s has stored P of block j.
+        for (int j = 0; ok && j < nb; ++j) {
+          if (!(ok = wait_v(cur))) break;
+          for (int s = 0; s < ns; ++s) {
+            if (!(ok = wait_p(s))) break;
+            values(s, j, cur.slot);
+          }
+          if (!ok) break;
+          if (release) commit(bar.v_empty(cur.slot));
+          cur.advance(R);
+        }
         if (!ok) break;
       }
       pos = cur;  // first event after this round (reuse: after the unit)
     }
   }
-  // Every tensor-core operation issued above must finish before the tensor
-  // memory is freed.
-  commit(bar.drain());
-  wait_drain(bar.drain(), 0u, kDrainLimitNs);
+  // Every tensor-core operation this warp issued must finish before the
+  // tensor memory is freed.
+  const uint32_t drain = bar.drain(score_warp ? 0 : 1);
+  commit(drain);
+  wait_drain(drain, 0u, kDrainLimitNs);
 }
 
 // ------------------------------------------------------------ softmax
@@ -628,7 +627,7 @@ template <int D>
 __device__ void softmax_role(const AttnParams& p, uint32_t tmem, const Barriers& bar,
                              volatile int* abort_flag, int warp, int lane) {
   using G = Geom<D>;
-  const int s = warp >> 2;  // Q slot of this warpgroup
+  const int s = (warp - kSoftmaxWarp0) >> 2;  // Q slot of this warpgroup
   const int quad = warp & 3;
   const int row_in_tile = quad * 32 + lane;
   const uint32_t lane_bits = static_cast<uint32_t>(quad * 32) << 16;
@@ -736,7 +735,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
       mbar_init(bar.v_full(i), 1);
       mbar_init(bar.v_empty(i), 1);
     }
-    mbar_init(bar.drain(), 1);
+    mbar_init(bar.drain(0), 1);
+    mbar_init(bar.drain(1), 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -761,16 +761,17 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
   if (warp == kLoadWarp) {
     load_role<D>(p, sQ, sK, sV, bar, abort_flag);
     __syncwarp();
-  } else if (warp == kMmaWarp) {
-    mma_role<D>(p, tmem, sQ, sK, sV, bar, abort_flag);
+  } else if (warp == kMmaWarp || warp == kPvWarp) {
+    mma_role<D>(p, tmem, sQ, sK, sV, bar, abort_flag, warp == kMmaWarp);
     __syncwarp();
-  } else if (warp < 8) {
+  } else if (warp >= kSoftmaxWarp0) {
     softmax_role<D>(p, tmem, bar, abort_flag, warp, lane);
     __syncwarp();
   }
 
   tc_fence_before();
   __syncthreads();
+  VLA_TRACE_END();
   if (warp == kMmaWarp) {
     tc_fence_after();
     tmem_dealloc(tmem, kTmemCols);
