@@ -29,10 +29,8 @@
 // row of block j in registers, so the tensor core computes S of block j+1
 // while block j is being exponentiated; P V of block j follows as soon as P
 // is stored.  A full round holds two Q tiles of one head (slots 0 and 1, one
-// per softmax warpgroup) and the two warpgroups take turns on the exp2 unit
-// (an mbarrier token passed back and forth) so the special-function pipe is
-// never contended by both at once.  A half round (the odd last tile of a
-// head) has slot 0 only.
+// per softmax warpgroup) whose exponentials share the special-function pipe.
+// A half round (the odd last tile of a head) has slot 0 only.
 //
 // Tensor memory (512 columns): slot s owns columns [256 s, 256 s + 256):
 // S at +0 (BK fp32 columns), O at +BK (DP = 64 or 80 fp32 columns), P at
@@ -68,7 +66,7 @@ constexpr int kSoftmaxWarp0 = 4;
 constexpr int kThreads = 384;
 constexpr int kMaxRing = 6;
 constexpr uint32_t kTmemCols = 512;
-constexpr int kNumBarriers = 14 + 4 * kMaxRing + 2;
+constexpr int kNumBarriers = 12 + 4 * kMaxRing + 2;
 constexpr uint32_t kBarrierRegionBytes = 512;  // barriers + tmem address + abort flag
 constexpr uint32_t kAlignSlack = 1024;
 constexpr unsigned long long kDrainLimitNs = 100000000ull;
@@ -77,7 +75,7 @@ constexpr unsigned long long kDrainLimitNs = 100000000ull;
 enum : int {
   kSiteLoadQ = 1, kSiteLoadK = 2, kSiteLoadV = 3,
   kSiteMmaQ = 11, kSiteMmaK = 12, kSiteMmaV = 13, kSiteMmaP = 14, kSiteMmaFree = 15,
-  kSiteSoftS = 21, kSiteSoftO = 22, kSiteSoftTok = 23,
+  kSiteSoftS = 21, kSiteSoftO = 22,
   kSiteDrain = 31,
 };
 
@@ -89,7 +87,7 @@ __device__ int g_vla_attn_status;  // 0 = ok, else 1000 + site of the first time
 enum : int {
   kTrMmaS = 1, kTrMmaPV = 2, kTrMmaSDone = 3, kTrMmaPVDone = 4, kTrMmaFree = 5, kTrMmaP = 6,
   kTrMmaV = 7, kTrMmaK = 8,
-  kTrSoftS = 10, kTrSoftMax = 11, kTrSoftTok = 12, kTrSoftExp = 13, kTrSoftP = 14,
+  kTrSoftS = 10, kTrSoftMax = 11, kTrSoftExp = 13, kTrSoftP = 14,
   kTrSoftEpi = 15,
 };
 #ifndef VLA_TRACE_EVENT
@@ -155,12 +153,11 @@ struct Barriers {
   __device__ uint32_t s_free(int s) const { return base + 8u * (6 + s); }   // S read out
   __device__ uint32_t p_full(int s) const { return base + 8u * (8 + s); }   // P in TMEM
   __device__ uint32_t o_prog(int s) const { return base + 8u * (10 + s); }  // each P V done
-  __device__ uint32_t tok(int s) const { return base + 8u * (12 + s); }     // exp2 turn
-  __device__ uint32_t k_full(int i) const { return base + 8u * (14 + i); }
-  __device__ uint32_t k_empty(int i) const { return base + 8u * (14 + kMaxRing + i); }
-  __device__ uint32_t v_full(int i) const { return base + 8u * (14 + 2 * kMaxRing + i); }
-  __device__ uint32_t v_empty(int i) const { return base + 8u * (14 + 3 * kMaxRing + i); }
-  __device__ uint32_t drain(int i) const { return base + 8u * (14 + 4 * kMaxRing + i); }
+  __device__ uint32_t k_full(int i) const { return base + 8u * (12 + i); }
+  __device__ uint32_t k_empty(int i) const { return base + 8u * (12 + kMaxRing + i); }
+  __device__ uint32_t v_full(int i) const { return base + 8u * (12 + 2 * kMaxRing + i); }
+  __device__ uint32_t v_empty(int i) const { return base + 8u * (12 + 3 * kMaxRing + i); }
+  __device__ uint32_t drain(int i) const { return base + 8u * (12 + 4 * kMaxRing + i); }
 };
 
 // Bounded wait for the phase of `bar` with the given parity, executed by a
@@ -502,8 +499,7 @@ struct SoftState {
 template <int D, int NC>
 __device__ __forceinline__ bool softmax_block(const AttnParams& p, SoftState& st, uint32_t tS,
                                               uint32_t tO, uint32_t tP, int nvalid, int j,
-                                              bool use_token, const Barriers& bar, int s,
-                                              uint32_t tok_parity, uint32_t o_parity,
+                                              const Barriers& bar, int s, uint32_t o_parity,
                                               volatile int* abort_flag, int lane) {
   using G = Geom<D>;
   const float c = p.c;
@@ -552,11 +548,6 @@ __device__ __forceinline__ bool softmax_block(const AttnParams& p, SoftState& st
   }
   const float mc = st.m_run * c;
   VLA_TRACE_EVENT(kTrSoftMax, s, j);
-  if (use_token) {
-    if (!wait_bounded(bar.tok(s), tok_parity, abort_flag, p.wait_limit_ns, kSiteSoftTok))
-      return false;
-  }
-  VLA_TRACE_EVENT(kTrSoftTok, s, j);
   float lsum[4] = {0.f, 0.f, 0.f, 0.f};
   uint32_t pk[64];
 #pragma unroll
@@ -568,10 +559,6 @@ __device__ __forceinline__ bool softmax_block(const AttnParams& p, SoftState& st
   }
 #pragma unroll
   for (int i = NC / 2; i < 64; ++i) pk[i] = 0u;
-  if (use_token) {
-    __syncwarp();
-    if (lane == 0) mbar_arrive(bar.tok(1 - s));
-  }
   VLA_TRACE_EVENT(kTrSoftExp, s, j);
   st.l_run += (lsum[0] + lsum[1]) + (lsum[2] + lsum[3]);
   if (j > 0) {
@@ -604,12 +591,10 @@ template <int D>
 __device__ __forceinline__ bool softmax_block_dispatch(const AttnParams& p, SoftState& st,
                                                        uint32_t tS, uint32_t tO, uint32_t tP,
                                                        int ncols, int nvalid, int j,
-                                                       bool use_token, const Barriers& bar,
-                                                       int s, uint32_t tp, uint32_t op,
+                                                       const Barriers& bar, int s, uint32_t op,
                                                        volatile int* abort_flag, int lane) {
-#define VLA_SB(NC)                                                                       \
-  return softmax_block<D, NC>(p, st, tS, tO, tP, nvalid, j, use_token, bar, s, tp, op, \
-                              abort_flag, lane)
+#define VLA_SB(NC) \
+  return softmax_block<D, NC>(p, st, tS, tO, tP, nvalid, j, bar, s, op, abort_flag, lane)
   if (ncols >= Geom<D>::BK) VLA_SB(Geom<D>::BK);
   switch (ncols) {
     case 112: VLA_SB(112);
@@ -635,9 +620,8 @@ __device__ void softmax_role(const AttnParams& p, uint32_t tmem, const Barriers&
   const uint32_t tO = tS + G::kColO;
   const uint32_t tP = tS + G::kColP;
   const int nb = p.num_kblocks;
-  uint32_t ns = 0;    // s_full phases consumed
-  uint32_t npv = 0;   // o_prog phases consumed
-  uint32_t ntok = 0;  // exp2 turns taken
+  uint32_t ns = 0;   // s_full phases consumed
+  uint32_t npv = 0;  // o_prog phases consumed
 
   for (int u = blockIdx.x; u < p.num_units; u += gridDim.x) {
     for (int rr = 0; rr < p.rounds_per_unit; ++rr) {
@@ -652,13 +636,10 @@ __device__ void softmax_role(const AttnParams& p, uint32_t tmem, const Barriers&
         ++ns;
         tc_fence_after();
         VLA_TRACE_EVENT(kTrSoftS, s, j);
-        // Slot 0 takes exp2 turns 0, 1, 2, ... right after slot 1's turns -1, 0, 1, ...
-        const uint32_t tp = s == 0 ? ((ntok & 1u) ^ 1u) : (ntok & 1u);
         const bool ok = softmax_block_dispatch<D>(
-            p, st, tS, tO, tP, block_cols<G::BK>(p.N, j), min(G::BK, p.N - j * G::BK), j, full,
-            bar, s, tp, (npv + j - 1) & 1u, abort_flag, lane);
+            p, st, tS, tO, tP, block_cols<G::BK>(p.N, j), min(G::BK, p.N - j * G::BK), j, bar, s,
+            (npv + j - 1) & 1u, abort_flag, lane);
         if (!ok) return;
-        if (full) ++ntok;
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(bar.p_full(s));
@@ -727,7 +708,6 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
       mbar_init(bar.s_free(s), 4);
       mbar_init(bar.p_full(s), 4);
       mbar_init(bar.o_prog(s), 1);
-      mbar_init(bar.tok(s), 4);
     }
     for (int i = 0; i < kMaxRing; ++i) {
       mbar_init(bar.k_full(i), 1);
