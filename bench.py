@@ -203,6 +203,22 @@ def run_reference(args, rank: int, world: int) -> None:
     print(json.dumps(line), flush=True)
 
 
+def max_over_ranks(values, world: int, device=None):
+    """Element-wise max of per-rank timings over all ranks (identity on one rank)."""
+    if world <= 1:
+        return [float(v) for v in values]
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(x) for x in t.tolist()]
+
+
+def rank_seed(rank: int) -> int:
+    """Seed of a rank's batch: every rank draws its own images (weak scaling)."""
+    return WORKLOAD.seed(0) + 7919 * rank
+
+
 # ---------------------------------------------------------------- CUDA path
 def run_ours(args, rank: int, world: int, local_rank: int) -> None:
     import torch
@@ -217,7 +233,7 @@ def run_ours(args, rank: int, world: int, local_rank: int) -> None:
         c = dataclasses.replace(c, B=int(args.images), name=f"{c.name}_B{int(args.images)}")
     stream = torch.cuda.current_stream(dev)
 
-    bits = si.packed_qkv(c.B, c.N, c.H, c.d, c.seed(0) + 7919 * rank)
+    bits = si.packed_qkv(c.B, c.N, c.H, c.d, rank_seed(rank))
     host_in = torch.from_numpy(bits.view(np.int16)).pin_memory()
     qkv = host_in.to(dev, non_blocking=False).view(torch.bfloat16)
     out = torch.empty((c.B, c.N, c.H, c.d), dtype=torch.bfloat16, device=dev)
@@ -280,10 +296,7 @@ def run_ours(args, rank: int, world: int, local_rank: int) -> None:
         barrier()
         e2e_ms = e0.elapsed_time(e1)
 
-    if world > 1:
-        t = torch.tensor([ms, e2e_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms, e2e_ms = float(t[0]), float(t[1])
+    ms, e2e_ms = max_over_ranks([ms, e2e_ms], world, dev)
 
     flops_call = float(c.flops())
     ms_step = ms / args.steps
