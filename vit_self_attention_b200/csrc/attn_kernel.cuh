@@ -548,15 +548,24 @@ __device__ __forceinline__ bool softmax_block(const AttnParams& p, SoftState& st
   }
   const float mc = st.m_run * c;
   VLA_TRACE_EVENT(kTrSoftMax, s, j);
-  float lsum[4] = {0.f, 0.f, 0.f, 0.f};
+  // Exponent arguments and running sums in packed fp32 pairs.
+  const uint64_t c2 = f32x2_pack(c, c);
+  const uint64_t nmc2 = f32x2_pack(-mc, -mc);
+  uint64_t acc2[2] = {0ull, 0ull};
   uint32_t pk[64];
 #pragma unroll
   for (int i = 0; i < NC / 2; ++i) {
-    const float p0 = ex2_approx(fmaf(x[2 * i], c, -mc));
-    const float p1 = ex2_approx(fmaf(x[2 * i + 1], c, -mc));
-    lsum[i & 3] += p0 + p1;
+    const uint64_t a = f32x2_fma(f32x2_pack(x[2 * i], x[2 * i + 1]), c2, nmc2);
+    float a0, a1;
+    f32x2_unpack(a, a0, a1);
+    const float p0 = ex2_approx(a0);
+    const float p1 = ex2_approx(a1);
+    acc2[i & 1] = f32x2_add(acc2[i & 1], f32x2_pack(p0, p1));
     pk[i] = pack_bf16x2(p0, p1);
   }
+  float lsum[4];
+  f32x2_unpack(acc2[0], lsum[0], lsum[1]);
+  f32x2_unpack(acc2[1], lsum[2], lsum[3]);
 #pragma unroll
   for (int i = NC / 2; i < 64; ++i) pk[i] = 0u;
   VLA_TRACE_EVENT(kTrSoftExp, s, j);
