@@ -120,6 +120,16 @@ uint64_t vla_attn_launch_count(void);
  */
 void vla_attn_set_wait_limit_ns(uint64_t ns);
 
+/*
+ * Testing hook: while `enable` is non-zero, launches that follow make every
+ * softmax warp wait on an mbarrier that nothing completes.  The wait runs out
+ * after the bound set with vla_attn_set_wait_limit_ns (default 1 s), the
+ * kernel records VLA_ATTN_ERR_TIMEOUT with site 41 and takes the error path
+ * described there; the output of such a launch is undefined.  No fault or
+ * trap is involved.  The attention pages describe no such hook.
+ */
+void vla_attn_set_test_stall(int enable);
+
 #ifdef __cplusplus
 }
 #endif

@@ -21,7 +21,7 @@ LIBRARY_PATH = os.path.join(_PKG, "libvla_attn.so")
 
 if not os.path.exists(LIBRARY_PATH):
     raise ImportError(
-        f"{LIBRARY_PATH} is missing: build it with `python -m vit_self_attention_b200.build` "
+        f"{LIBRARY_PATH} is missing: build it with `python vit_self_attention_b200/build.py` "
         "(nvcc, sm_100a); there is no fallback implementation")
 
 _lib = ctypes.CDLL(LIBRARY_PATH)
@@ -44,6 +44,8 @@ _lib.vla_attn_launch_count.argtypes = []
 _lib.vla_attn_launch_count.restype = ctypes.c_uint64
 _lib.vla_attn_set_wait_limit_ns.argtypes = [ctypes.c_uint64]
 _lib.vla_attn_set_wait_limit_ns.restype = None
+_lib.vla_attn_set_test_stall.argtypes = [_I]
+_lib.vla_attn_set_test_stall.restype = None
 
 # Status codes of include/vla_attn.h
 OK = 0
@@ -61,6 +63,7 @@ EXPORTED_SYMBOLS = (
     "vla_attn_fwd", "vla_attn_fwd_host", "vla_attn_strerror", "vla_attn_last_device_status",
     "vla_attn_reset_device_status", "vla_attn_max_tokens", "vla_attn_launch_count",
     "vla_attn_set_wait_limit_ns",
+    "vla_attn_set_test_stall",
 )
 
 
@@ -136,6 +139,11 @@ def vla_attn_set_wait_limit_ns(ns: int) -> None:
     _lib.vla_attn_set_wait_limit_ns(int(ns))
 
 
+def vla_attn_set_test_stall(enable: bool) -> None:
+    """Testing hook: following launches wait on a barrier nothing completes (see the header)."""
+    _lib.vla_attn_set_test_stall(1 if enable else 0)
+
+
 def attention(qkv, scale: float | None = None, out=None, stream=None):
     """Convenience wrapper for a contiguous bf16 CUDA tensor ``qkv`` of shape
     ``[B, N, 3, H, d]``; returns ``out`` (allocated by torch if None) ``[B, N, H, d]``."""
@@ -158,5 +166,5 @@ def attention(qkv, scale: float | None = None, out=None, stream=None):
 __all__ = [
     "LIBRARY_PATH", "EXPORTED_SYMBOLS", "VlaAttnError", "vla_attn_fwd", "vla_attn_fwd_host",
     "vla_attn_strerror", "vla_attn_last_device_status", "vla_attn_reset_device_status",
-    "vla_attn_max_tokens", "vla_attn_launch_count", "vla_attn_set_wait_limit_ns", "attention",
+    "vla_attn_max_tokens", "vla_attn_launch_count", "vla_attn_set_wait_limit_ns", "vla_attn_set_test_stall", "attention",
 ]

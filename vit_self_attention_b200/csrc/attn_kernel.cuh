@@ -66,7 +66,7 @@ constexpr int kSoftmaxWarp0 = 4;
 constexpr int kThreads = 384;
 constexpr int kMaxRing = 6;
 constexpr uint32_t kTmemCols = 512;
-constexpr int kNumBarriers = 12 + 4 * kMaxRing + 2;
+constexpr int kNumBarriers = 12 + 4 * kMaxRing + 3;
 constexpr uint32_t kBarrierRegionBytes = 512;  // barriers + tmem address + abort flag
 constexpr uint32_t kAlignSlack = 1024;
 constexpr unsigned long long kDrainLimitNs = 100000000ull;
@@ -77,6 +77,7 @@ enum : int {
   kSiteMmaQ = 11, kSiteMmaK = 12, kSiteMmaV = 13, kSiteMmaP = 14, kSiteMmaFree = 15,
   kSiteSoftS = 21, kSiteSoftO = 22,
   kSiteDrain = 31,
+  kSiteTestStall = 41,
 };
 
 __device__ int g_vla_attn_status;  // 0 = ok, else 1000 + site of the first timed-out wait
@@ -137,6 +138,7 @@ struct AttnParams {
   int reuse;               // 1 when num_kblocks <= ring: a unit loads its K/V once
   float c;                 // scale * log2(e)
   unsigned long long wait_limit_ns;
+  int test_stall;          // testing hook: softmax warps wait on a barrier nothing completes
 };
 
 template <int D>
@@ -158,6 +160,8 @@ struct Barriers {
   __device__ uint32_t v_full(int i) const { return base + 8u * (12 + 2 * kMaxRing + i); }
   __device__ uint32_t v_empty(int i) const { return base + 8u * (12 + 3 * kMaxRing + i); }
   __device__ uint32_t drain(int i) const { return base + 8u * (12 + 4 * kMaxRing + i); }
+  // Never arrived at: the testing hook's wait runs out on it.
+  __device__ uint32_t never() const { return base + 8u * (12 + 4 * kMaxRing + 2); }
 };
 
 // Bounded wait for the phase of `bar` with the given parity, executed by a
@@ -631,6 +635,12 @@ __device__ void softmax_role(const AttnParams& p, uint32_t tmem, const Barriers&
   const int nb = p.num_kblocks;
   uint32_t ns = 0;   // s_full phases consumed
   uint32_t npv = 0;  // o_prog phases consumed
+  if (p.test_stall) {
+    // Testing hook: a wait that nothing completes runs out after the bound,
+    // which takes the whole CTA down the error path.
+    (void)wait_bounded(bar.never(), 0u, abort_flag, p.wait_limit_ns, kSiteTestStall);
+    return;
+  }
 
   for (int u = blockIdx.x; u < p.num_units; u += gridDim.x) {
     for (int rr = 0; rr < p.rounds_per_unit; ++rr) {
@@ -726,6 +736,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
     }
     mbar_init(bar.drain(0), 1);
     mbar_init(bar.drain(1), 1);
+    mbar_init(bar.never(), 1);
     *abort_flag = 0;
     fence_mbar_init();
   }

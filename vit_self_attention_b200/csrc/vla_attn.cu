@@ -23,6 +23,7 @@ constexpr int kMaxDevices = 64;
 
 std::atomic<uint64_t> g_launches{0};
 std::atomic<unsigned long long> g_wait_limit_ns{0};
+std::atomic<int> g_test_stall{0};
 
 struct DriverFns {
   PFN_cuTensorMapEncodeTiled_v12000 encode = nullptr;
@@ -213,6 +214,7 @@ int launch(const void* q, void* o, int B, int N, int H, float scale, cudaStream_
   prm.c = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
   const unsigned long long lim = g_wait_limit_ns.load();
   prm.wait_limit_ns = lim == 0 ? kDefaultWaitLimitNs : lim;
+  prm.test_stall = g_test_stall.load();
 
   rc = ensure_smem_attr<D>(dev, static_cast<int>(smem));
   if (rc != VLA_ATTN_OK) return rc;
@@ -328,5 +330,7 @@ int vla_attn_max_tokens(int d) { return (d == 64 || d == 72) ? kMaxTokens : 0; }
 uint64_t vla_attn_launch_count(void) { return g_launches.load(); }
 
 void vla_attn_set_wait_limit_ns(uint64_t ns) { g_wait_limit_ns.store(ns); }
+
+void vla_attn_set_test_stall(int enable) { g_test_stall.store(enable ? 1 : 0); }
 
 }  // extern "C"
