@@ -6,6 +6,7 @@ shape).  One step = one call of the fused attention kernel over the whole
 batch.  Prints ONE JSON line (rank 0).
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+  python bench.py --configs     # per-config report (one JSON line per item, 1 GPU)
 
 Under torchrun every rank runs the same per-GPU batch on its own GPU (weak
 scaling, no collective on the data path); the elapsed time is the max over
@@ -341,6 +342,152 @@ def run_ours(args, rank: int, world: int, local_rank: int) -> None:
     print(json.dumps(line), flush=True)
 
 
+def _percentile(xs, q):
+    xs = sorted(xs)
+    return xs[min(len(xs) - 1, int(round(q * (len(xs) - 1))))]
+
+
+def run_configs(args) -> None:
+    """Per-config report on one GPU: warm (back-to-back calls in a CUDA graph) and
+    cold-L2 (after a 256 MB write) per-call time (median, P95)
+    and roofline fraction for every workload, the L-layer sequence replayed from one
+    CUDA graph with fresh buffers per layer (configs 1-4), longer sequences
+    (384 px and 448 px ViT-L/14 grids), and the fp64 oracle on all host cores and
+    on one core."""
+    import torch
+
+    import oracle
+    import vit_self_attention_b200 as vab
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    peaks = measured_peaks()
+    p_bf16 = float(peaks.get("bf16_tflops", 1590.0)) * 1e12
+    hbm = float(peaks.get("hbm_gbs", 6650.0)) * 1e9
+    scratch = torch.empty(256 << 20, dtype=torch.uint8, device=dev)  # > L2 (126 MB)
+
+    def buffers(c, bits):
+        qkv = torch.from_numpy(bits.view(np.int16)).to(dev).view(torch.bfloat16)
+        out = torch.empty((c.B, c.N, c.H, c.d), dtype=torch.bfloat16, device=dev)
+        return qkv, out
+
+    def call(c, qkv, out):
+        b = qkv.data_ptr()
+        st = c.H * c.d * 2
+        vab.vla_attn_fwd(b, b + st, b + 2 * st, out, c.B, c.N, c.H, c.d, c.scale)
+
+    def timed(c, qkv, out, iters, flush):
+        ts = []
+        for i in range(iters):
+            if flush:
+                scratch.fill_(i & 0xFF)
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record()
+            call(c, qkv, out)
+            e1.record()
+            e1.synchronize()
+            ts.append(e0.elapsed_time(e1) * 1e3)  # us
+        return ts
+
+    items = [(c, True) for c in si.CONFIGS] + [
+        (si.AttnConfig(6, "vit_l14_384px_b64", 64, 730, 16, 64, 0.125, 1.0, 1.0, 1, 24), False),
+        (si.AttnConfig(7, "vit_l14_448px_b64", 64, 1025, 16, 64, 0.125, 1.0, 1.0, 1, 24), False)]
+    for c, std in items:
+        bits = c.qkv(0) if std else si.packed_qkv(c.B, c.N, c.H, c.d, 4242 + c.N)
+        qkv, out = buffers(c, bits)
+        for _ in range(10):
+            call(c, qkv, out)
+        torch.cuda.synchronize()
+        iters = 20 if c.B * c.N >= 100000 else 100
+        # Warm: 20 back-to-back calls on the same buffers in one CUDA graph, so the
+        # host-side cost of a call (argument checks, tensor-map encoding) does not
+        # leave the GPU idle between calls; per-call time = replay time / 20.
+        side = torch.cuda.Stream(dev)
+        side.wait_stream(torch.cuda.current_stream(dev))
+        with torch.cuda.stream(side):
+            call(c, qkv, out)
+        torch.cuda.current_stream(dev).wait_stream(side)
+        torch.cuda.synchronize()
+        g20 = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g20, stream=side):
+            for _ in range(20):
+                call(c, qkv, out)
+        for _ in range(3):
+            g20.replay()
+        torch.cuda.synchronize()
+        warm = []
+        for _ in range(max(5, iters // 20)):
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record()
+            g20.replay()
+            e1.record()
+            e1.synchronize()
+            warm.append(e0.elapsed_time(e1) * 1e3 / 20)
+        del g20
+        # Cold L2: a 256 MB write before each call; the call is enqueued while that
+        # write runs, so the events bracket the kernel alone.
+        cold = timed(c, qkv, out, min(iters, 50), True)
+        flops, nbytes = c.flops(), c.bytes()
+        t_roof = max(flops / p_bf16, nbytes / hbm) * 1e6
+        rec = {"mode": "configs", "workload": c.name, "B": c.B, "N": c.N, "H": c.H, "d": c.d,
+               "bound": "tensor" if flops / p_bf16 > nbytes / hbm else "hbm",
+               "roofline_us": t_roof,
+               "warm_us": {"median": statistics.median(warm), "p95": _percentile(warm, 0.95)},
+               "cold_l2_us": {"median": statistics.median(cold), "p95": _percentile(cold, 0.95)},
+               "tflops_warm": flops / statistics.median(warm) / 1e6,
+               "frac_warm": t_roof / statistics.median(warm),
+               "frac_cold_l2": t_roof / statistics.median(cold)}
+        if std and c.layers > 1 and c.B * c.N < 100000:
+            # L layers, each with its own input and output buffers, in one graph.
+            layers = [buffers(c, c.qkv(i % c.calls)) for i in range(c.layers)]
+            side = torch.cuda.Stream(dev)
+            side.wait_stream(torch.cuda.current_stream(dev))
+            with torch.cuda.stream(side):
+                for q_, o_ in layers:
+                    call(c, q_, o_)
+            torch.cuda.current_stream(dev).wait_stream(side)
+            torch.cuda.synchronize()
+            graph = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(graph, stream=side):
+                for q_, o_ in layers:
+                    call(c, q_, o_)
+            for _ in range(5):
+                graph.replay()
+            torch.cuda.synchronize()
+            reps = []
+            for _ in range(50):
+                e0 = torch.cuda.Event(enable_timing=True)
+                e1 = torch.cuda.Event(enable_timing=True)
+                e0.record()
+                graph.replay()
+                e1.record()
+                e1.synchronize()
+                reps.append(e0.elapsed_time(e1) * 1e3)
+            t = statistics.median(reps)
+            rec["graph_layers"] = c.layers
+            rec["graph_us"] = {"median": t, "p95": _percentile(reps, 0.95),
+                               "per_layer": t / c.layers}
+            rec["graph_images_per_s"] = c.B / (t * 1e-6)
+            rec["graph_frac"] = t_roof * c.layers / t
+            del graph, layers
+        print(json.dumps(rec), flush=True)
+        del qkv, out
+        torch.cuda.empty_cache()
+
+    c = WORKLOAD
+    bits = si.packed_qkv(1, c.N, c.H, c.d, c.seed(0))
+    flops1 = 4.0 * c.H * c.N * c.N * c.d
+    for threads in (oracle.default_threads(), 1):
+        t0 = time.perf_counter()
+        oracle.attention_packed_bf16(bits, c.scale, threads=threads)
+        dt = time.perf_counter() - t0
+        print(json.dumps({"mode": "configs", "oracle": "fp64 C++", "cores": threads,
+                          "sample": f"1 image x {c.H} heads of {c.name}",
+                          "seconds": dt, "tflops": flops1 / dt / 1e12}), flush=True)
+
+
 def main() -> None:
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -353,7 +500,12 @@ def main() -> None:
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end leg")
     ap.add_argument("--images", type=int, default=None,
                     help="override B (profiling captures of a smaller case of the same kernel)")
+    ap.add_argument("--configs", action="store_true",
+                    help="per-config report instead of the benchmark line (1 GPU)")
     args = ap.parse_args()
+    if args.configs:
+        run_configs(args)
+        return
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))

@@ -68,7 +68,11 @@ typedef enum {
  *   o        device pointer to [B, N, H, d] bf16 output, 16-byte aligned; must
  *            not overlap the input.
  *   B        images (camera views x batch), >= 1.
- *   N        tokens per image (patches + CLS), 1 <= N <= vla_attn_max_tokens(d).
+ *   N        tokens per image (patches + CLS), 1 <= N <= vla_attn_max_tokens(d)
+ *            (16384).  Up to 768 tokens for d=64 (560 for d=72) a head's K and
+ *            V stay in shared memory for all its query tiles; longer sequences
+ *            stream K/V blocks through the shared-memory ring per pair of
+ *            query tiles (same result, more L2 traffic).
  *   H        heads, >= 1.
  *   d        head dimension, 64 (ViT-B/16, ViT-L/14) or 72 (SigLIP-So400m/14).
  *   scale    logit scale, usually 1/sqrt(d); finite and > 0.

@@ -66,7 +66,7 @@ def test_argument_validation_on_host():
     assert call(N=-5) == vab.ERR_SHAPE
     assert call(d=128, k=Q + H * 128 * 2, v=Q + 4 * H * 128) == vab.ERR_UNSUPPORTED
     assert call(d=32, k=Q + H * 32 * 2, v=Q + 4 * H * 32) == vab.ERR_UNSUPPORTED
-    assert call(N=578) == vab.ERR_UNSUPPORTED
+    assert call(N=16385) == vab.ERR_UNSUPPORTED
     assert call(k=K + 2) == vab.ERR_SHAPE          # not the packed relation
     assert call(v=K) == vab.ERR_SHAPE
     assert call(q=Q + 2, k=K + 2, v=V + 2) == vab.ERR_ALIGN
@@ -92,7 +92,7 @@ def test_strerror_and_limits():
     for st in range(-9, 1):
         assert vab.vla_attn_strerror(st)
     assert "unknown" in vab.vla_attn_strerror(-99)
-    assert vab.vla_attn_max_tokens(64) == 577 and vab.vla_attn_max_tokens(72) == 577
+    assert vab.vla_attn_max_tokens(64) == 16384 and vab.vla_attn_max_tokens(72) == 16384
     assert vab.vla_attn_max_tokens(128) == 0
 
 

@@ -43,11 +43,48 @@ def test_edge_token_counts(N, d):
     assert_parity(got, want, f"B={B} N={N} H={H} d={d}")
 
 
-@pytest.mark.parametrize("B,H,N,d", [(160, 1, 197, 64), (10, 16, 257, 64), (12, 13, 577, 64),
+# Longer sequences (384 px and 448 px ViT/14 grids and beyond): K/V resident while a
+# head's blocks fit the ring (d=64: N <= 768, d=72: N <= 560), streamed per round after.
+LONG_N = [578, 640, 641, 729, 730, 768, 769, 1025, 2049]
+
+
+@pytest.mark.parametrize("d", [64, 72])
+@pytest.mark.parametrize("N", LONG_N)
+def test_long_sequences(N, d):
+    B, H = 1, 2
+    bits = si.packed_qkv(B, N, H, d, seed=90000 + 10 * N + d)
+    scale = 1.0 / math.sqrt(d)
+    want = oracle.attention_packed_bf16(bits, scale)
+    got = run_cuda(bits, scale)
+    assert_parity(got, want, f"B={B} N={N} H={H} d={d}")
+
+
+def test_longest_sequence_sampled_rows():
+    """N = 16384 (the accepted maximum), one head per image, rows sampled across all
+    128 query tiles, against the oracle computed row by row."""
+    B, N, H, d = 2, 16384, 1, 64
+    bits = si.packed_qkv(B, N, H, d, seed=91234)
+    scale = 0.125
+    import vit_self_attention_b200 as vab
+    out = vab.attention(device_qkv(bits), scale)
+    torch.cuda.synchronize()
+    rng = np.random.default_rng(11)
+    rows = [(b, 0, n) for b in range(B) for n in (0, 1, 127, 128, 8191, 8192, N - 2, N - 1)]
+    rows += [(int(rng.integers(0, B)), 0, int(rng.integers(0, N))) for _ in range(120)]
+    want = oracle.attention_rows_packed_bf16(bits, scale, rows)
+    idx = torch.tensor(rows, dtype=torch.long, device="cuda")
+    got = out[idx[:, 0], idx[:, 2], idx[:, 1]].float().cpu().numpy().astype(np.float64)
+    assert_parity(got, want, "B=2 N=16384 H=1 sampled rows")
+
+
+@pytest.mark.parametrize("B,H,N,d", [(8, 4, 577, 64), (4, 5, 1025, 64), (6, 5, 600, 72),
+                                     (160, 1, 197, 64), (10, 16, 257, 64), (12, 13, 577, 64),
                                      (75, 2, 577, 72), (1, 1, 577, 64), (148, 1, 129, 72),
                                      (300, 1, 50, 64)])
 def test_schedules(B, H, N, d):
-    """Whole-head work units (B*H >= #SMs) and per-round units, persistent multi-unit CTAs."""
+    """Whole-head work units (B*H >= #SMs), per-round units (fewer heads, more tiles than
+    SMs; includes K/V streaming at N > 768 / d=72 N > 560), single-tile units (all tiles
+    fit on the SMs), and persistent multi-unit CTAs."""
     bits = si.packed_qkv(B, N, H, d, seed=90000 + B * 7 + H * 3 + N + d)
     scale = 1.0 / math.sqrt(d)
     want = oracle.attention_packed_bf16(bits, scale)
@@ -197,6 +234,7 @@ def test_rejects_host_and_short_buffers():
     st = vab.vla_attn_fwd(fb, fb + H * d * 2, fb + 2 * H * d * 2, fb, B, N, H, d, 0.125,
                           check=False)
     assert st == vab.ERR_MEMORY  # output overlapping the input
-    assert vab.vla_attn_fwd(fb, fb + H * d * 2, fb + 2 * H * d * 2, out, B, 578, H, d, 0.125,
+    assert vab.vla_attn_fwd(fb, fb + H * d * 2, fb + 2 * H * d * 2, out, B,
+                            vab.vla_attn_max_tokens(d) + 1, H, d, 0.125,
                             check=False) == vab.ERR_UNSUPPORTED
     assert vab.vla_attn_launch_count() >= 0

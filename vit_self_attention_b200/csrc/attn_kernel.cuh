@@ -132,6 +132,8 @@ struct AttnParams {
   int num_qtiles;          // ceil(N / 128)
   int rounds_per_head;     // ceil(num_qtiles / 2): a round = up to two Q tiles
   int rounds_per_unit;     // rounds_per_head (whole head) or 1
+  int tile_units;          // 1: a unit is one Q tile (slot 0 only), for batches whose
+                           // tiles all fit on the SMs at once
   int units_per_head;
   int num_units;
   int ring;                // K/V ring slots (<= kMaxRing)
@@ -212,8 +214,9 @@ __device__ __forceinline__ int block_cols(int N, int j) {
 
 // One (unit, round) step of the schedule, identical for every role.
 struct Round {
-  int b, h, r;  // image, head, round index within the head
-  int nslots;   // 2 = full round (tiles 2r, 2r+1), 1 = half round (tile 2r only)
+  int b, h, r;  // image, head, round index within the head (tile index for tile units)
+  int t0;       // Q tile of slot 0 (slot 1 has t0 + 1)
+  int nslots;   // 2 = full round (tiles 2r, 2r+1), 1 = half round or a tile unit
   bool first;   // first round of its unit
   bool last;    // last round of its unit
 };
@@ -224,7 +227,13 @@ __device__ __forceinline__ Round make_round(const AttnParams& p, int u, int rr) 
   x.r = (u % p.units_per_head) * p.rounds_per_unit + rr;
   x.b = bh / p.H;
   x.h = bh % p.H;
-  x.nslots = (2 * x.r + 1 < p.num_qtiles) ? 2 : 1;
+  if (p.tile_units) {
+    x.t0 = x.r;
+    x.nslots = 1;
+  } else {
+    x.t0 = 2 * x.r;
+    x.nslots = (2 * x.r + 1 < p.num_qtiles) ? 2 : 1;
+  }
   x.first = rr == 0;
   x.last = rr == p.rounds_per_unit - 1;
   return x;
@@ -262,7 +271,7 @@ __device__ void load_role(const AttnParams& p, uint32_t sQ, uint32_t sK, uint32_
       return false;
     if (elect_one()) {
       const uint32_t dst = sQ + s * G::kQBytes;
-      const int row0 = (2 * x.r + s) * kQRows;
+      const int row0 = (x.t0 + s) * kQRows;
       mbar_arrive_expect_tx(bar.q_full(s), G::kQBytes);
       tma_load_5d(dst, &p.tm_q, bar.q_full(s), 0, x.h, 0, row0, x.b);
       if (G::kHasTail)
@@ -647,7 +656,7 @@ __device__ void softmax_role(const AttnParams& p, uint32_t tmem, const Barriers&
       const Round x = make_round(p, u, rr);
       const bool full = x.nslots == 2;
       if (!full && s == 1) continue;
-      const int tile = 2 * x.r + s;
+      const int tile = x.t0 + s;
       SoftState st{-INFINITY, 0.0f};
       for (int j = 0; j < nb; ++j) {
         if (!wait_bounded(bar.s_full(s), ns & 1u, abort_flag, p.wait_limit_ns, kSiteSoftS))

@@ -17,7 +17,11 @@
 
 namespace {
 
-constexpr int kMaxTokens = 577;  // 576 patches + CLS: ViT-L/14 at 336 x 336
+// Longest sequence accepted.  577 (ViT-L/14 at 336 px) keeps a head's K/V
+// resident in shared memory for all its query tiles; longer sequences (e.g.
+// 730 at 384 px, 1025 at 448 px) stream K/V through the ring per round of two
+// query tiles once a head's blocks exceed it (d=64: N > 768; d=72: N > 560).
+constexpr int kMaxTokens = 16384;
 constexpr unsigned long long kDefaultWaitLimitNs = 1000000000ull;
 constexpr int kMaxDevices = 64;
 
@@ -202,10 +206,14 @@ int launch(const void* q, void* o, int B, int N, int H, float scale, cudaStream_
   prm.H = H;
   prm.num_kblocks = nb;
   prm.num_qtiles = nq;
+  // Work units: whole heads (K/V loaded once per head) when there are enough
+  // heads to fill the SMs; otherwise single Q tiles if all of them fit on the
+  // SMs at once (shortest per-CTA chain), else single rounds of two tiles.
   prm.rounds_per_head = (nq + 1) / 2;
   const long long heads = static_cast<long long>(B) * H;
   prm.rounds_per_unit = heads >= di.sm_count ? prm.rounds_per_head : 1;
-  prm.units_per_head = prm.rounds_per_head / prm.rounds_per_unit;
+  prm.tile_units = (heads < di.sm_count && nq > 1 && heads * nq <= di.sm_count) ? 1 : 0;
+  prm.units_per_head = prm.tile_units ? nq : prm.rounds_per_head / prm.rounds_per_unit;
   const long long units = heads * prm.units_per_head;
   if (units > 0x7FFFFFFFll) return VLA_ATTN_ERR_SHAPE;
   prm.num_units = static_cast<int>(units);
