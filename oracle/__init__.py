@@ -1,11 +1,13 @@
-"""fp64 CPU oracle for the ViT/SigLIP self-attention core -- TEST INFRASTRUCTURE.
+"""fp64 CPU oracle for the ViT/SigLIP self-attention core and the LayerNorm and
+linear layers around it -- TEST INFRASTRUCTURE.
 
 Only the tests, ``__graft_entry__.smoke()`` and the benchmark's CPU-baseline
 leg use this package.  The CUDA library neither imports nor links it, and it
 imports nothing from the CUDA package.
 
-The arithmetic lives in ``vla_attn_oracle.cpp`` (plain definition of
-``O = softmax(Q K^T * scale) V`` per image and head, fp64 throughout); this
+The arithmetic lives in ``vla_attn_oracle.cpp`` (plain definitions of
+``O = softmax(Q K^T * scale) V`` per image and head, of LayerNorm over the last
+dimension and of ``x @ w.T + bias (+ res)``, fp64 throughout); this
 module only marshals numpy arrays through ctypes.  ``OracleLib`` can wrap any
 build of that source (the tests compile deliberately broken copies to show
 that the pins catch them); the module-level functions use the real build.
@@ -33,6 +35,11 @@ class OracleLib:
 
     def __init__(self, path: str):
         lib = ctypes.CDLL(path)
+        lib.oracle_layernorm_bf16.argtypes = [_U16P, _U16P, _U16P, _DP, _I, _I,
+                                              ctypes.c_double, _I]
+        lib.oracle_layernorm_bf16.restype = _I
+        lib.oracle_linear_bf16.argtypes = [_U16P, _U16P, _U16P, _U16P, _DP, _I, _I, _I, _I]
+        lib.oracle_linear_bf16.restype = _I
         lib.oracle_attn_f64.argtypes = [_DP, _DP, _DP, _DP, _I, _I, _I, _I, ctypes.c_double, _I]
         lib.oracle_attn_f64.restype = _I
         lib.oracle_attn_probs_f64.argtypes = [_DP, _DP, _DP, _I, _I, _I, _I, ctypes.c_double]
@@ -109,6 +116,44 @@ class OracleLib:
         return out
 
 
+    def layernorm_bf16(self, x_bits, gamma_bits, beta_bits, eps: float,
+                       threads: int = 0) -> np.ndarray:
+        """fp64 LayerNorm over the last dimension of bf16 ``x`` (``[..., W]``)."""
+        x = np.ascontiguousarray(x_bits, dtype=np.uint16)
+        W = int(x.shape[-1])
+        M = int(x.size // W)
+        g = np.ascontiguousarray(gamma_bits, dtype=np.uint16).reshape(W)
+        b = np.ascontiguousarray(beta_bits, dtype=np.uint16).reshape(W)
+        out = np.empty(x.shape, dtype=np.float64)
+        rc = self._lib.oracle_layernorm_bf16(_ptr(x, ctypes.c_uint16), _ptr(g, ctypes.c_uint16),
+                                             _ptr(b, ctypes.c_uint16), _ptr(out, ctypes.c_double),
+                                             M, W, float(eps), int(threads))
+        if rc != 0:
+            raise ValueError(f"oracle_layernorm_bf16 rejected the input (rc={rc})")
+        return out
+
+    def linear_bf16(self, x_bits, w_bits, bias_bits=None, res_bits=None,
+                    threads: int = 0) -> np.ndarray:
+        """fp64 ``x @ w.T + bias (+ res)`` for bf16 ``x [..., K]``, ``w [N, K]``."""
+        x = np.ascontiguousarray(x_bits, dtype=np.uint16)
+        w = np.ascontiguousarray(w_bits, dtype=np.uint16)
+        N, K = (int(v) for v in w.shape)
+        if x.shape[-1] != K:
+            raise ValueError("x and w disagree on K")
+        M = int(x.size // K)
+        b = None if bias_bits is None else np.ascontiguousarray(bias_bits, dtype=np.uint16).reshape(N)
+        r = None if res_bits is None else np.ascontiguousarray(res_bits, dtype=np.uint16).reshape(M, N)
+        out = np.empty(x.shape[:-1] + (N,), dtype=np.float64)
+        rc = self._lib.oracle_linear_bf16(
+            _ptr(x, ctypes.c_uint16), _ptr(w, ctypes.c_uint16),
+            None if b is None else _ptr(b, ctypes.c_uint16),
+            None if r is None else _ptr(r, ctypes.c_uint16), _ptr(out, ctypes.c_double),
+            M, K, N, int(threads))
+        if rc != 0:
+            raise ValueError(f"oracle_linear_bf16 rejected the input (rc={rc})")
+        return out
+
+
 _default: OracleLib | None = None
 
 
@@ -140,7 +185,16 @@ def attention_rows_packed_bf16(qkv_bits, scale: float, rows, threads: int = 0) -
     return lib().attention_rows_packed_bf16(qkv_bits, scale, rows, threads)
 
 
+def layernorm_bf16(x_bits, gamma_bits, beta_bits, eps: float, threads: int = 0) -> np.ndarray:
+    return lib().layernorm_bf16(x_bits, gamma_bits, beta_bits, eps, threads)
+
+
+def linear_bf16(x_bits, w_bits, bias_bits=None, res_bits=None, threads: int = 0) -> np.ndarray:
+    return lib().linear_bf16(x_bits, w_bits, bias_bits, res_bits, threads)
+
+
 SOURCE = _build.SRC
 
 __all__ = ["OracleLib", "lib", "attention_f64", "probs_f64", "attention_packed_bf16",
-           "attention_rows_packed_bf16", "default_threads", "SOURCE"]
+           "attention_rows_packed_bf16", "layernorm_bf16", "linear_bf16", "default_threads",
+           "SOURCE"]

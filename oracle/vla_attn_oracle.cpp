@@ -227,4 +227,67 @@ int oracle_attn_rows_packed_bf16(const uint16_t* qkv, int B, int N, int H, int d
   return 0;
 }
 
+// ---------------------------------------------------------------------------
+// The two operations on either side of the attention core in a ViT block, in
+// the same plain fp64 style (test infrastructure only, like the rest):
+//
+//   LayerNorm over the last dimension (width W) of every row m:
+//     mu  = (1/W) sum_i x[m,i]
+//     var = (1/W) sum_i (x[m,i] - mu)^2                (biased, as LayerNorm)
+//     y[m,i] = (x[m,i] - mu) / sqrt(var + eps) * gamma[i] + beta[i]
+//   "FluxVLA docs, inference acceleration", Triton fused kernels (norm
+//   fusion: residual add + LayerNorm in one kernel); the ViT block applies it
+//   before its qkv linear.
+//
+//   Linear layer with bias and optional residual (weight stored [N, K] as in
+//   nn.Linear, i.e. the pages' weight(K,N) transposed):
+//     y[m,n] = sum_k x[m,k] * w[n,k] + bias[n] + res[m,n]
+//   same page, section 3, CUDA custom operators: cublasLt fused GEMM + bias
+//   (+ residual), D = inp @ weight + bias (+ res); "Pi0 VLA deployment
+//   tutorial", section 3.2: the block's qkv linear feeds the attention.
+//
+// bf16 inputs are widened exactly; bias and res may be null (treated as 0).
+
+// LayerNorm of M rows of width W (bf16 x, gamma, beta) into fp64 y.
+int oracle_layernorm_bf16(const uint16_t* x, const uint16_t* gamma, const uint16_t* beta,
+                          double* y, int M, int W, double eps, int nthreads) {
+  if (M < 0 || W <= 0 || !(eps >= 0.0)) return -1;
+  parallel_for(static_cast<long>(M), nthreads, [&](long m) {
+    const uint16_t* xm = x + m * static_cast<std::ptrdiff_t>(W);
+    double sum = 0.0;
+    for (int i = 0; i < W; ++i) sum += widen_bf16(xm[i]);
+    const double mu = sum / W;
+    double ss = 0.0;
+    for (int i = 0; i < W; ++i) {
+      const double dv = widen_bf16(xm[i]) - mu;
+      ss += dv * dv;
+    }
+    const double var = ss / W;
+    const double rstd = 1.0 / std::sqrt(var + eps);
+    double* ym = y + m * static_cast<std::ptrdiff_t>(W);
+    for (int i = 0; i < W; ++i)
+      ym[i] = (widen_bf16(xm[i]) - mu) * rstd * widen_bf16(gamma[i]) + widen_bf16(beta[i]);
+  });
+  return 0;
+}
+
+// y[m,n] = sum_k x[m,k] w[n,k] + bias[n] + res[m,n]  (bf16 inputs, fp64 y).
+int oracle_linear_bf16(const uint16_t* x, const uint16_t* w, const uint16_t* bias,
+                       const uint16_t* res, double* y, int M, int K, int N, int nthreads) {
+  if (M < 0 || K <= 0 || N <= 0) return -1;
+  parallel_for(static_cast<long>(M), nthreads, [&](long m) {
+    std::vector<double> xm(static_cast<size_t>(K));
+    for (int k = 0; k < K; ++k) xm[k] = widen_bf16(x[m * static_cast<std::ptrdiff_t>(K) + k]);
+    for (int n = 0; n < N; ++n) {
+      const uint16_t* wn = w + n * static_cast<std::ptrdiff_t>(K);
+      double acc = 0.0;
+      for (int k = 0; k < K; ++k) acc += xm[k] * widen_bf16(wn[k]);
+      if (bias != nullptr) acc += widen_bf16(bias[n]);
+      if (res != nullptr) acc += widen_bf16(res[m * static_cast<std::ptrdiff_t>(N) + n]);
+      y[m * static_cast<std::ptrdiff_t>(N) + n] = acc;
+    }
+  });
+  return 0;
+}
+
 }  // extern "C"

@@ -95,6 +95,15 @@ def bf16_bits_to_f32(bits: np.ndarray) -> np.ndarray:
     return (b.astype(np.uint32) << np.uint32(16)).view(np.float32)
 
 
+def normal_bf16(seed: int, shape, mean: float = 0.0, std: float = 1.0) -> np.ndarray:
+    """bf16 bit patterns (``uint16``, given shape) of ``mean + std * N(0, 1)`` draws from the
+    counter-based generator, in memory order (fp64 draw, fp32 scale, bf16 round)."""
+    count = int(np.prod(shape))
+    z = normals(seed, 0, count)
+    v = (np.float64(mean) + np.float64(std) * z).astype(np.float32)
+    return f32_to_bf16_bits(v).reshape(shape)
+
+
 def _fill_chunk(out: np.ndarray, seed: int, start: int, count: int, H: int, d: int,
                 sigma_qk: float, sigma_v: float) -> None:
     z = normals(seed, start, count)

@@ -8,9 +8,12 @@ them against the real oracle; ``test_oracle_mutants`` runs them against
 deliberately broken copies of the oracle source and requires each copy to fail
 at least one pin.
 
-Definition being pinned (multi-head self-attention of the ViT block, as in the
+Definitions being pinned (multi-head self-attention of the ViT block, as in the
 Pi0 Flash Attention tutorial, sections 1 and 3.2):
-``o[b,i,h,:] = sum_j softmax_j(scale * q[b,i,h,:] . k[b,j,h,:]) v[b,j,h,:]``.
+``o[b,i,h,:] = sum_j softmax_j(scale * q[b,i,h,:] . k[b,j,h,:]) v[b,j,h,:]``;
+and the layers around it: LayerNorm over the last dimension and the linear layer
+``x @ w.T + bias (+ res)`` (FluxVLA inference-acceleration page: norm fusion,
+and section 3's cublasLt fused GEMM + bias (+ residual)).
 """
 from __future__ import annotations
 
@@ -248,6 +251,146 @@ def pin_rows_entry(lib):
         _close(got[r_], full[b, n, h], 0.0, f"row {(b, h, n)}")
 
 
+# --------------------------------------------------------------- LayerNorm
+# y[m,i] = (x[m,i] - mean_m) / sqrt(var_m + eps) * gamma[i] + beta[i], biased variance
+# ("FluxVLA docs, inference acceleration", Triton fused kernels: norm fusion).
+
+def _bits(a):
+    """Exact bf16 bit patterns of values that bf16 represents exactly."""
+    a = np.asarray(a, dtype=np.float32)
+    bits = si.f32_to_bf16_bits(a)
+    assert np.array_equal(si.bf16_bits_to_f32(bits), a), "value not exact in bf16"
+    return bits
+
+
+def _bf16(a):
+    return si.f32_to_bf16_bits(np.asarray(a, dtype=np.float32))
+
+
+def pin_layernorm_closed_forms(lib):
+    """Constant rows give beta; a row of +a / -a gives +-a/sqrt(a^2 + eps) * gamma + beta;
+    with gamma = 1, beta = 0 every row has mean 0 and variance var / (var + eps)."""
+    W = 12
+    gamma = _bf16(np.linspace(0.5, 2.0, W))
+    beta = _bf16(np.linspace(-1.0, 1.0, W))
+    x = _bits(np.full((3, W), [[2.0], [-7.5], [0.0]]))
+    y = lib.layernorm_bf16(x, gamma, beta, 1e-6)
+    _close(y, np.broadcast_to(si.bf16_bits_to_f32(beta), (3, W)), 0.0, "constant rows -> beta")
+    a, eps = 3.0, 0.25
+    row = np.array([a if i % 2 == 0 else -a for i in range(W)])
+    y = lib.layernorm_bf16(_bits(row[None]), gamma, beta, eps)[0]
+    want = row / math.sqrt(a * a + eps) * si.bf16_bits_to_f32(gamma) + si.bf16_bits_to_f32(beta)
+    _close(y, want, 1e-12, "two-valued row")
+    one, zero = _bits(np.ones(64)), _bits(np.zeros(64))
+    x = _bf16(_rng(3).normal(0.4, 1.7, size=(5, 64)))
+    eps = 0.5
+    y = lib.layernorm_bf16(x, one, zero, eps)
+    xv = si.bf16_bits_to_f32(x).astype(np.float64)
+    var = xv.var(axis=1)
+    _close(y.mean(axis=1), np.zeros(5), 1e-12, "output mean")
+    _close(y.var(axis=1), var / (var + eps), 1e-12, "output variance")
+
+
+def pin_layernorm_shift_invariance(lib):
+    """With eps = 0 the result ignores a constant shift and a positive scale of the row
+    (values chosen exactly representable after the shift and scale)."""
+    W = 32
+    gamma = _bf16(_rng(4).normal(size=W))
+    beta = _bf16(_rng(5).normal(size=W))
+    base = _rng(6).integers(-40, 40, size=(4, W)).astype(np.float64)
+    y0 = lib.layernorm_bf16(_bits(base), gamma, beta, 0.0)
+    y1 = lib.layernorm_bf16(_bits(base + 24.0), gamma, beta, 0.0)
+    y2 = lib.layernorm_bf16(_bits(base * 4.0), gamma, beta, 0.0)
+    _close(y1, y0, 1e-12, "shift")
+    _close(y2, y0, 1e-12, "scale")
+
+
+def pin_layernorm_brute_force_and_torch(lib):
+    """Pure-Python loops on tiny rows, and torch's fp64 layer_norm on a ViT-width batch."""
+    import torch
+    W, M, eps = 7, 3, 1e-5
+    x = _bf16(_rng(7).normal(size=(M, W)))
+    g = _bf16(_rng(8).normal(size=W))
+    b = _bf16(_rng(9).normal(size=W))
+    xv, gv, bv = (si.bf16_bits_to_f32(t).astype(float).tolist() for t in (x, g, b))
+    want = []
+    for r in xv:
+        mu = sum(r) / W
+        var = sum((v - mu) ** 2 for v in r) / W
+        want.append([(r[i] - mu) / math.sqrt(var + eps) * gv[i] + bv[i] for i in range(W)])
+    _close(lib.layernorm_bf16(x, g, b, eps), np.array(want), 1e-12, "brute-force LayerNorm")
+    W, M = 768, 40
+    x = _bf16(_rng(10).normal(0.1, 1.3, size=(M, W)))
+    g = _bf16(_rng(11).normal(1.0, 0.2, size=W))
+    b = _bf16(_rng(12).normal(0.0, 0.2, size=W))
+    tw = lambda t: torch.from_numpy(si.bf16_bits_to_f32(t).astype(np.float64))
+    want = torch.nn.functional.layer_norm(tw(x), (W,), tw(g), tw(b), 1e-6).numpy()
+    _close(lib.layernorm_bf16(x, g, b, 1e-6), want, 1e-10, "torch layer_norm fp64")
+
+
+# ------------------------------------------------------------------ linear
+# y[m,n] = sum_k x[m,k] w[n,k] + bias[n] + res[m,n]  (same page, section 3: cublasLt
+# fused GEMM + bias (+ residual); the Pi0 tutorial's qkv linear feeds attention).
+
+def pin_linear_closed_forms(lib):
+    """Identity weights return x + bias, zero weights return bias, a rank-1 weight
+    u v^T returns (x . v) u + bias, and a residual is added once."""
+    K = 16
+    x = _bf16(_rng(13).normal(size=(6, K)))
+    xv = si.bf16_bits_to_f32(x).astype(np.float64)
+    bias = _bf16(_rng(14).normal(size=K))
+    bv = si.bf16_bits_to_f32(bias).astype(np.float64)
+    _close(lib.linear_bf16(x, _bits(np.eye(K)), bias), xv + bv, 1e-12, "identity weight")
+    _close(lib.linear_bf16(x, _bits(np.zeros((5, K))), bias[:5]), np.broadcast_to(bv[:5], (6, 5)),
+           0.0, "zero weight")
+    u = np.array([1.0, -2.0, 0.5, 4.0, 0.25])
+    v = _rng(15).integers(-3, 4, size=K).astype(np.float64)
+    w = _bits(np.outer(u, v))
+    _close(lib.linear_bf16(x, w), np.outer(xv @ v, u), 1e-12, "rank-1 weight")
+    res = _bf16(_rng(16).normal(size=(6, 5)))
+    rv = si.bf16_bits_to_f32(res).astype(np.float64)
+    w = _bf16(_rng(17).normal(size=(5, K)))
+    _close(lib.linear_bf16(x, w, bias[:5], res) - lib.linear_bf16(x, w, bias[:5]), rv, 1e-12,
+           "residual")
+
+
+def pin_linear_permutation_and_linearity(lib):
+    """A permutation weight permutes the input features; the map is linear in x."""
+    K = 24
+    perm = _rng(18).permutation(K)
+    P = np.zeros((K, K))
+    P[np.arange(K), perm] = 1.0
+    x = _bf16(_rng(19).normal(size=(3, K)))
+    xv = si.bf16_bits_to_f32(x).astype(np.float64)
+    _close(lib.linear_bf16(x, _bits(P)), xv[:, perm], 0.0, "permutation weight")
+    w = _bf16(_rng(20).normal(size=(9, K)))
+    a = _rng(21).integers(-8, 8, size=(4, K)).astype(np.float64)
+    b = _rng(22).integers(-8, 8, size=(4, K)).astype(np.float64)
+    _close(lib.linear_bf16(_bits(a + b), w),
+           lib.linear_bf16(_bits(a), w) + lib.linear_bf16(_bits(b), w), 1e-9, "linearity")
+
+
+def pin_linear_brute_force_and_torch(lib):
+    """Pure-Python loops on a tiny case (weights [N, K] as nn.Linear stores them), and
+    torch's fp64 addmm on the ViT-B/16 qkv shape."""
+    import torch
+    M, K, N = 3, 5, 4
+    x = _bf16(_rng(23).normal(size=(M, K)))
+    w = _bf16(_rng(24).normal(size=(N, K)))
+    b = _bf16(_rng(25).normal(size=N))
+    xv, wv, bv = (si.bf16_bits_to_f32(t).astype(float).tolist() for t in (x, w, b))
+    want = [[sum(xv[m][k] * wv[n][k] for k in range(K)) + bv[n] for n in range(N)]
+            for m in range(M)]
+    _close(lib.linear_bf16(x, w, b), np.array(want), 1e-12, "brute-force linear")
+    M, K, N = 50, 768, 2304
+    x = _bf16(_rng(26).normal(size=(M, K)))
+    w = _bf16(_rng(27).normal(size=(N, K)) / math.sqrt(K))
+    b = _bf16(_rng(28).normal(size=N))
+    tw = lambda t: torch.from_numpy(si.bf16_bits_to_f32(t).astype(np.float64))
+    want = torch.addmm(tw(b), tw(x), tw(w).T).numpy()
+    _close(lib.linear_bf16(x, w, b), want, 1e-10, "torch addmm fp64")
+
+
 ALL_PINS = [
     pin_golden_closed_forms,
     pin_single_token,
@@ -262,4 +405,10 @@ ALL_PINS = [
     pin_torch_sdpa_configs,
     pin_d72_zero_padding,
     pin_rows_entry,
+    pin_layernorm_closed_forms,
+    pin_layernorm_shift_invariance,
+    pin_layernorm_brute_force_and_torch,
+    pin_linear_closed_forms,
+    pin_linear_permutation_and_linearity,
+    pin_linear_brute_force_and_torch,
 ]

@@ -33,6 +33,25 @@ MUTANTS = [
      "const uint16_t* row = qkv + (b * N + n) * tok;"),
     ("weights_not_exponentiated_in_probs", "for (int j = 0; j < N; ++j) probs[j] = s[j] / l;",
      "for (int j = 0; j < N; ++j) probs[j] = s[j];"),
+    ("ln_unbiased_variance", "const double var = ss / W;", "const double var = ss / (W - 1);"),
+    ("ln_eps_dropped", "const double rstd = 1.0 / std::sqrt(var + eps);",
+     "const double rstd = 1.0 / std::sqrt(var);"),
+    ("ln_beta_dropped",
+     "ym[i] = (widen_bf16(xm[i]) - mu) * rstd * widen_bf16(gamma[i]) + widen_bf16(beta[i]);",
+     "ym[i] = (widen_bf16(xm[i]) - mu) * rstd * widen_bf16(gamma[i]);"),
+    ("ln_mean_not_subtracted",
+     "ym[i] = (widen_bf16(xm[i]) - mu) * rstd * widen_bf16(gamma[i]) + widen_bf16(beta[i]);",
+     "ym[i] = widen_bf16(xm[i]) * rstd * widen_bf16(gamma[i]) + widen_bf16(beta[i]);"),
+    ("linear_weight_transposed",
+     "const uint16_t* wn = w + n * static_cast<std::ptrdiff_t>(K);\n      double acc = 0.0;\n"
+     "      for (int k = 0; k < K; ++k) acc += xm[k] * widen_bf16(wn[k]);",
+     "double acc = 0.0;\n"
+     "      for (int k = 0; k < K; ++k) acc += xm[k] * widen_bf16(w[k * static_cast<std::ptrdiff_t>(N) + n]);"),
+    ("linear_bias_dropped", "if (bias != nullptr) acc += widen_bf16(bias[n]);", ""),
+    ("linear_last_k_dropped", "for (int k = 0; k < K; ++k) acc += xm[k] * widen_bf16(wn[k]);",
+     "for (int k = 0; k < K - 1; ++k) acc += xm[k] * widen_bf16(wn[k]);"),
+    ("linear_residual_dropped",
+     "if (res != nullptr) acc += widen_bf16(res[m * static_cast<std::ptrdiff_t>(N) + n]);", ""),
 ]
 
 
