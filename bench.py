@@ -7,6 +7,7 @@ batch.  Prints ONE JSON line (rank 0).
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
   python bench.py --configs     # per-config report (one JSON line per item, 1 GPU)
+  python bench.py --block       # LayerNorm / linear layers and the attention half-block
 
 Under torchrun every rank runs the same per-GPU batch on its own GPU (weak
 scaling, no collective on the data path); the elapsed time is the max over
@@ -488,6 +489,120 @@ def run_configs(args) -> None:
                           "seconds": dt, "tflops": flops1 / dt / 1e12}), flush=True)
 
 
+def _graph_time_us(fn, reps: int = 20, iters: int = 10) -> list[float]:
+    """Per-call times (us) of ``fn`` captured ``reps`` times back to back in one CUDA
+    graph, over ``iters`` replays (the host cost of a call does not idle the GPU)."""
+    import torch
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        fn()
+    torch.cuda.current_stream().wait_stream(side)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=side):
+        for _ in range(reps):
+            fn()
+    for _ in range(2):
+        g.replay()
+    torch.cuda.synchronize()
+    out = []
+    for _ in range(iters):
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record()
+        g.replay()
+        e1.record()
+        e1.synchronize()
+        out.append(e0.elapsed_time(e1) * 1e3 / reps)
+    del g
+    return out
+
+
+def run_block(args) -> None:
+    """LayerNorm and the linear layers (qkv projection; output projection with the
+    residual add) on the encoder shapes and the bench batch, and the attention half of
+    a ViT block (LayerNorm -> qkv -> attention -> output projection + residual): one
+    layer at the bench batch, and the L-layer sequence for the encoder workloads."""
+    import math as _m
+
+    import torch
+
+    import vit_self_attention_b200 as vab
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    peaks = measured_peaks()
+    p_bf16 = float(peaks["bf16_tflops"]) * 1e12
+    hbm = float(peaks["hbm_gbs"]) * 1e9
+    ws = torch.empty(vab.vla_linear_workspace_bytes(), dtype=torch.uint8, device=dev)
+
+    def t_(shape, mean=0.0, std=1.0, seed=1):
+        b = si.normal_bf16(seed, shape, mean, std)
+        return torch.from_numpy(b.view(np.int16)).to(dev).view(torch.bfloat16)
+
+    for c in list(si.CONFIGS[1:4]) + [si.CONFIGS[4]]:
+        W = c.H * c.d
+        M = c.B * c.N
+        x = t_((c.B, c.N, W), 0.0, 1.0, 11)
+        g, be = t_((W,), 1.0, 0.1, 12), t_((W,), 0.0, 0.1, 13)
+        wq, bq = t_((3 * W, W), 0.0, 1.0 / _m.sqrt(W), 14), t_((3 * W,), 0.0, 0.1, 15)
+        wo, bo = t_((W, W), 0.0, 1.0 / _m.sqrt(W), 16), t_((W,), 0.0, 0.1, 17)
+        xn = torch.empty_like(x)
+        qkv = torch.empty((c.B, c.N, 3 * W), dtype=torch.bfloat16, device=dev)
+        o = torch.empty((c.B, c.N, c.H, c.d), dtype=torch.bfloat16, device=dev)
+        y = torch.empty_like(x)
+        ln = lambda: vab.layernorm(x, g, be, 1e-6, out=xn)
+        lq = lambda: vab.linear(xn, wq, bq, out=qkv, workspace=ws)
+        at = lambda: vab.attention(qkv.view(c.B, c.N, 3, c.H, c.d), c.scale, out=o)
+        lo = lambda: vab.linear(o.view(c.B, c.N, W), wo, bo, x, out=y, workspace=ws)
+        ref = lambda: torch.addmm(bq, xn.view(M, W), wq.t(), out=qkv.view(M, 3 * W))
+        big = c.B * c.N >= 100000
+        reps, iters = (3, 5) if big else (20, 10)
+        med = lambda f: statistics.median(_graph_time_us(f, reps, iters))
+        t_ln, t_q, t_at, t_o, t_ref = med(ln), med(lq), med(at), med(lo), med(ref)
+        fq, fo = 2.0 * M * W * 3 * W, 2.0 * M * W * W
+        rec = {"mode": "block", "workload": c.name, "tokens": M, "width": W,
+               "layernorm": {"us": t_ln, "gbs": 4.0 * M * W / t_ln / 1e3,
+                             "frac_hbm": 4.0 * M * W / t_ln / 1e-6 / hbm},
+               "qkv_linear": {"us": t_q, "tflops": fq / t_q / 1e6,
+                              "frac_bf16": fq / t_q / 1e-6 / p_bf16,
+                              "torch_addmm_us": t_ref},
+               "attention": {"us": t_at, "tflops": c.flops() / t_at / 1e6},
+               "out_linear_residual": {"us": t_o, "tflops": fo / t_o / 1e6,
+                                       "frac_bf16": fo / t_o / 1e-6 / p_bf16}}
+        chain = lambda: (ln(), lq(), at(), lo())
+        t_chain = med(chain)
+        rec["half_block_us"] = t_chain
+        rec["half_block_tflops"] = (fq + fo + c.flops()) / t_chain / 1e6
+        if not big:
+            # The encoder's L layers (fresh weights and activations per layer) in one graph.
+            layers = []
+            for i in range(c.layers):
+                layers.append((t_((W,), 1.0, 0.1, 100 + 7 * i), t_((W,), 0.0, 0.1, 101 + 7 * i),
+                               t_((3 * W, W), 0.0, 1.0 / _m.sqrt(W), 102 + 7 * i),
+                               t_((3 * W,), 0.0, 0.1, 103 + 7 * i),
+                               t_((W, W), 0.0, 1.0 / _m.sqrt(W), 104 + 7 * i),
+                               t_((W,), 0.0, 0.1, 105 + 7 * i)))
+            xs = [x.clone() for _ in range(c.layers + 1)]
+
+            def encoder():
+                for i, (g_, b_, wq_, bq_, wo_, bo_) in enumerate(layers):
+                    vab.layernorm(xs[i], g_, b_, 1e-6, out=xn)
+                    vab.linear(xn, wq_, bq_, out=qkv, workspace=ws)
+                    vab.attention(qkv.view(c.B, c.N, 3, c.H, c.d), c.scale, out=o)
+                    vab.linear(o.view(c.B, c.N, W), wo_, bo_, xs[i], out=xs[i + 1], workspace=ws)
+
+            t_enc = statistics.median(_graph_time_us(encoder, 1, 20))
+            rec["encoder_layers"] = c.layers
+            rec["encoder_half_blocks_us"] = t_enc
+            rec["encoder_images_per_s"] = c.B / (t_enc * 1e-6)
+            del layers, xs
+        print(json.dumps(rec), flush=True)
+        del x, xn, qkv, o, y, wq, wo
+        torch.cuda.empty_cache()
+
+
 def main() -> None:
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -502,9 +617,14 @@ def main() -> None:
                     help="override B (profiling captures of a smaller case of the same kernel)")
     ap.add_argument("--configs", action="store_true",
                     help="per-config report instead of the benchmark line (1 GPU)")
+    ap.add_argument("--block", action="store_true",
+                    help="LayerNorm / linear layers and the attention half-block (1 GPU)")
     args = ap.parse_args()
     if args.configs:
         run_configs(args)
+        return
+    if args.block:
+        run_block(args)
         return
 
     world = int(os.environ.get("WORLD_SIZE", "1"))

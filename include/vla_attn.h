@@ -41,6 +41,7 @@
 #ifndef VLA_ATTN_H_
 #define VLA_ATTN_H_
 
+#include <stddef.h>
 #include <stdint.h>
 
 #ifdef __cplusplus
@@ -133,6 +134,52 @@ void vla_attn_set_wait_limit_ns(uint64_t ns);
  * trap is involved.  The attention pages describe no such hook.
  */
 void vla_attn_set_test_stall(int enable);
+
+/*
+ * LayerNorm over the last dimension of M rows of width W (the norm before a
+ * ViT block's qkv linear; "FluxVLA docs, inference acceleration", Triton fused
+ * kernels: norm fusion):
+ *   y[m,i] = (x[m,i] - mean_m) / sqrt(var_m + eps) * gamma[i] + beta[i],
+ *   var_m the biased variance, statistics in fp32.
+ *   x, y     device pointers, [M, W] bf16 row-major, 16-byte aligned; y may be
+ *            x (in place) but must not otherwise overlap an input.
+ *   gamma, beta  device pointers, [W] bf16, 16-byte aligned.
+ *   W        a multiple of 8, at most 2048 (ViT-B 768, ViT-L 1024, SigLIP 1152).
+ *   eps      finite, >= 0 (timm ViT and SigLIP use 1e-6).
+ * Returns VLA_ATTN_OK or a negative status (same codes as vla_attn_fwd;
+ * VLA_ATTN_ERR_SCALE for a bad eps).
+ */
+int vla_layernorm_fwd(const void* x, const void* gamma, const void* beta, void* y, int M, int W,
+                      float eps, void* stream);
+
+/*
+ * Linear layer with bias and optional residual, weights in nn.Linear layout
+ * (same page, section 3, CUDA custom operators: cublasLt fused GEMM + bias
+ * (+ residual), one launch; the "Pi0 VLA deployment tutorial", section 3.2:
+ * the block's qkv linear feeds the attention):
+ *   y[m,n] = sum_k x[m,k] * w[n,k] + bias[n] + res[m,n]
+ * Runs one cuBLASLt matmul (bf16 in, fp32 accumulate, bf16 out, bias in the
+ * epilogue, res as C with beta = 1).  For the qkv linear (N = 3 H d), y is the
+ * packed [B, tokens, 3, H, d] input of vla_attn_fwd.
+ *   x        device, [M, K] bf16 row-major.
+ *   w        device, [N, K] bf16 row-major.
+ *   bias     device [N] bf16, or NULL (no bias).
+ *   res      device [M, N] bf16, or NULL (no residual); may equal y.
+ *   y        device, [M, N] bf16 row-major; must not overlap x, w, bias, the
+ *            workspace, or res unless it is res.
+ *   K, N     multiples of 8.  All pointers 16-byte aligned.
+ *   workspace, workspace_bytes  caller-owned device scratch for cuBLASLt
+ *            (vla_linear_workspace_bytes() recommended; NULL with 0 allowed);
+ *            the library allocates nothing.  Calls that share a workspace
+ *            must be ordered on one stream.
+ * Returns VLA_ATTN_OK or a negative status (VLA_ATTN_ERR_CUDA if cuBLASLt
+ * fails or finds no algorithm).
+ */
+int vla_linear_fwd(const void* x, const void* w, const void* bias, const void* res, void* y,
+                   int M, int K, int N, void* workspace, size_t workspace_bytes, void* stream);
+
+/* Recommended workspace size for vla_linear_fwd (bytes). */
+size_t vla_linear_workspace_bytes(void);
 
 #ifdef __cplusplus
 }

@@ -38,3 +38,24 @@ def assert_parity(got: np.ndarray, want: np.ndarray, what: str,
     mx, mean = errors(got, want)
     assert mx <= max_tol and mean <= mean_tol, (
         f"{what}: max|err| {mx:.3e} (tol {max_tol:.0e}), mean|err| {mean:.3e} (tol {mean_tol:.0e})")
+
+
+def assert_close_bf16(got: np.ndarray, want: np.ndarray, what: str, mag=None) -> None:
+    """Tolerance of a bf16 output layer derived from its arithmetic (LayerNorm, linear):
+    fp32 accumulation, then bf16 round-to-nearest, possibly twice (the GEMM + bias term,
+    then the sum with the residual), each rounding at most 2^-9 of the magnitude it rounds.
+    Elementwise |err| <= 2^-7 mag + 2^-9 with mag = |want| or, with a residual, the sum of
+    the magnitudes of the two terms; the mean error at most 2^-8 of the mean magnitude
+    (plus 1e-4)."""
+    got = np.asarray(got, dtype=np.float64)
+    want = np.asarray(want, dtype=np.float64)
+    assert got.shape == want.shape, f"{what}: shape {got.shape} vs {want.shape}"
+    assert np.all(np.isfinite(got)), f"{what}: non-finite outputs"
+    err = np.abs(got - want)
+    mag = np.abs(want) if mag is None else np.asarray(mag, dtype=np.float64)
+    bound = 2.0 ** -7 * mag + 2.0 ** -9
+    worst = float(np.max(err - bound))
+    mean_err, mean_mag = float(err.mean()), float(mag.mean())
+    assert worst <= 0.0, f"{what}: an element exceeds 2^-7|y| + 2^-9 by {worst:.3e}"
+    assert mean_err <= 2.0 ** -8 * mean_mag + 1e-4, (
+        f"{what}: mean|err| {mean_err:.3e} vs mean|y| {mean_mag:.3e}")

@@ -15,7 +15,7 @@ def declared_functions():
     with open(HEADER) as f:
         text = f.read()
     text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
-    return sorted(set(re.findall(r"\b(vla_attn_[a-z_]+)\s*\(", text)))
+    return sorted(set(re.findall(r"\b(vla_[a-z_]+)\s*\(", text)))
 
 
 def test_header_declares_the_entry_points():
@@ -116,3 +116,33 @@ def test_product_package_has_no_oracle_or_fallback():
             assert "oracle" not in src.lower(), f"{fn} mentions the oracle"
             assert "scaled_dot_product_attention" not in src, f"{fn} has a torch attention path"
             assert "softmax(" not in src.replace("softmax(Q", "").replace("softmax(q", ""), fn
+
+
+def test_layernorm_and_linear_validation_on_host():
+    """The LayerNorm and linear entry points reject bad arguments before touching a GPU."""
+    import math as _m
+
+    import vit_self_attention_b200 as vab
+    X, G, B_, Y = 0x10000000, 0x11000000, 0x12000000, 0x13000000
+
+    def ln(x=X, g=G, b=B_, y=Y, M=4, W=768, eps=1e-6):
+        return vab.vla_layernorm_fwd(x, g, b, y, M, W, eps, stream=0, check=False)
+
+    assert ln(x=None) == vab.ERR_NULL and ln(g=None) == vab.ERR_NULL and ln(y=None) == vab.ERR_NULL
+    assert ln(M=0) == vab.ERR_SHAPE and ln(W=0) == vab.ERR_SHAPE
+    assert ln(W=12) == vab.ERR_UNSUPPORTED and ln(W=2056) == vab.ERR_UNSUPPORTED
+    assert ln(eps=-1.0) == vab.ERR_SCALE and ln(eps=_m.nan) == vab.ERR_SCALE
+    assert ln(x=X + 2) == vab.ERR_ALIGN and ln(b=B_ + 8) == vab.ERR_ALIGN
+
+    W_, BI, R, WS = 0x14000000, 0x15000000, 0x16000000, 0x17000000
+
+    def lin(x=X, w=W_, bias=BI, res=R, y=Y, M=4, K=768, N=2304, ws=WS, wsb=1 << 20):
+        return vab.vla_linear_fwd(x, w, bias, res, y, M, K, N, ws, wsb, stream=0, check=False)
+
+    assert lin(x=None) == vab.ERR_NULL and lin(w=None) == vab.ERR_NULL
+    assert lin(y=None) == vab.ERR_NULL and lin(ws=None) == vab.ERR_NULL
+    assert lin(M=0) == vab.ERR_SHAPE and lin(K=-8) == vab.ERR_SHAPE
+    assert lin(K=12) == vab.ERR_UNSUPPORTED and lin(N=10) == vab.ERR_UNSUPPORTED
+    assert lin(bias=BI + 2) == vab.ERR_ALIGN and lin(res=R + 4) == vab.ERR_ALIGN
+    assert lin(ws=WS + 8) == vab.ERR_ALIGN
+    assert vab.vla_linear_workspace_bytes() >= 1 << 20

@@ -1,0 +1,189 @@
+"""LayerNorm and linear layers around the attention core vs. the fp64 oracle.
+
+Stage-wise: every GPU stage is compared with the oracle on identical bf16 inputs
+(the GPU's own bf16 output of the previous stage feeds the oracle's next stage).
+Tolerance: the attention stage keeps the attention bound (max |err| <= 2e-2,
+mean |err| <= 2e-3); LayerNorm and linear outputs use the bound derived from their
+arithmetic (bf16 rounding of an fp32 result, possibly twice -- GEMM + bias, then the
+residual sum -- each at most 2^-9 of what it rounds: elementwise
+|err| <= 2^-7 (|x w^T + b| + |res|) + 2^-9, mean error <= 2^-8 of the mean magnitude),
+since their outputs reach |y| ~ 6 where one bf16 ulp is 0.03.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import seeded_inputs as si
+from gpu_helpers import assert_close_bf16, assert_parity, needs_gpu
+
+pytestmark = [pytest.mark.gpu, needs_gpu]
+
+# (name, B, N, H, d): the encoder workloads; width W = H d, tokens M = B N.
+ENCODERS = [(c.name, c.B, c.N, c.H, c.d) for c in si.CONFIGS[:4]]
+
+
+def dev(bits):
+    return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).cuda().view(torch.bfloat16)
+
+
+def host(t):
+    return t.contiguous().view(torch.int16).cpu().numpy().view(np.uint16)
+
+
+def f64(t):
+    return t.float().cpu().numpy().astype(np.float64)
+
+
+def ln_inputs(M, W, seed):
+    return (si.normal_bf16(seed, (M, W), 0.2, 1.3), si.normal_bf16(seed + 1, (W,), 1.0, 0.1),
+            si.normal_bf16(seed + 2, (W,), 0.0, 0.1))
+
+
+def linear_inputs(M, K, N, seed):
+    return (si.normal_bf16(seed, (M, K)), si.normal_bf16(seed + 1, (N, K), 0.0, 1.0 / math.sqrt(K)),
+            si.normal_bf16(seed + 2, (N,), 0.0, 0.1))
+
+
+@pytest.mark.parametrize("name,B,N,H,d", ENCODERS)
+def test_layernorm_encoder_widths(name, B, N, H, d):
+    import vit_self_attention_b200 as vab
+    M, W = B * N, H * d
+    x, g, b = ln_inputs(M, W, 100 + W)
+    got = vab.layernorm(dev(x), dev(g), dev(b), 1e-6)
+    torch.cuda.synchronize()
+    assert_close_bf16(f64(got), oracle.layernorm_bf16(x, g, b, 1e-6), f"LayerNorm {name}")
+
+
+@pytest.mark.parametrize("M,W", [(1, 8), (7, 16), (33, 248), (5, 256), (9, 264), (3, 2048),
+                                 (1000, 768)])
+def test_layernorm_edge_shapes_and_in_place(M, W):
+    import vit_self_attention_b200 as vab
+    x, g, b = ln_inputs(M, W, 200 + M + W)
+    want = oracle.layernorm_bf16(x, g, b, 1e-5)
+    xt = dev(x)
+    got = vab.layernorm(xt, dev(g), dev(b), 1e-5)
+    torch.cuda.synchronize()
+    assert_close_bf16(f64(got), want, f"LayerNorm M={M} W={W}")
+    vab.layernorm(xt, dev(g), dev(b), 1e-5, out=xt)  # in place
+    torch.cuda.synchronize()
+    assert_close_bf16(f64(xt), want, f"LayerNorm in place M={M} W={W}")
+
+
+@pytest.mark.parametrize("name,B,N,H,d", ENCODERS)
+def test_qkv_linear_encoder_shapes(name, B, N, H, d):
+    import vit_self_attention_b200 as vab
+    M, K = B * N, H * d
+    x, w, b = linear_inputs(M, K, 3 * K, 300 + K)
+    got = vab.linear(dev(x), dev(w), dev(b))
+    torch.cuda.synchronize()
+    assert_close_bf16(f64(got), oracle.linear_bf16(x, w, b), f"qkv linear {name}")
+
+
+@pytest.mark.parametrize("M,K,N,bias,res", [(1, 8, 8, True, False), (5, 16, 24, False, False),
+                                            (129, 768, 768, True, True), (77, 64, 200, False, True),
+                                            (1000, 1024, 1024, True, True)])
+def test_linear_bias_residual_variants(M, K, N, bias, res):
+    import vit_self_attention_b200 as vab
+    x, w, b = linear_inputs(M, K, N, 400 + M + K + N)
+    r = si.normal_bf16(500 + M, (M, N)) if res else None
+    got = vab.linear(dev(x), dev(w), dev(b) if bias else None, dev(r) if res else None)
+    torch.cuda.synchronize()
+    want = oracle.linear_bf16(x, w, b if bias else None, r)
+    assert_close_bf16(f64(got), want, f"linear M={M} K={K} N={N} bias={bias} res={res}",
+                      mag=residual_magnitude(x, w, b if bias else None, r))
+
+
+def test_linear_in_place_residual():
+    """y = x @ w.T + bias + y (the output projection adding into the residual stream)."""
+    import vit_self_attention_b200 as vab
+    M, K = 591, 768
+    x, w, b = linear_inputs(M, K, K, 600)
+    r = si.normal_bf16(601, (M, K))
+    rt = dev(r)
+    vab.linear(dev(x), dev(w), dev(b), rt, out=rt)
+    torch.cuda.synchronize()
+    assert_close_bf16(f64(rt), oracle.linear_bf16(x, w, b, r), "in-place residual",
+                      mag=residual_magnitude(x, w, b, r))
+
+
+def residual_magnitude(x, w, b, r):
+    """|x @ w.T + b| + |r|: the magnitudes the two roundings of a residual linear act on."""
+    if r is None:
+        return np.abs(oracle.linear_bf16(x, w, b))
+    return np.abs(oracle.linear_bf16(x, w, b)) + np.abs(si.bf16_bits_to_f32(r).astype(np.float64))
+
+
+def block_weights(W, seed):
+    return {"g": si.normal_bf16(seed, (W,), 1.0, 0.1), "be": si.normal_bf16(seed + 1, (W,), 0.0, 0.1),
+            "wqkv": si.normal_bf16(seed + 2, (3 * W, W), 0.0, 1.0 / math.sqrt(W)),
+            "bqkv": si.normal_bf16(seed + 3, (3 * W,), 0.0, 0.1),
+            "wo": si.normal_bf16(seed + 4, (W, W), 0.0, 1.0 / math.sqrt(W)),
+            "bo": si.normal_bf16(seed + 5, (W,), 0.0, 0.1)}
+
+
+@pytest.mark.parametrize("cfg", [0, 1, 3])
+def test_attention_half_block_stagewise(cfg):
+    """x -> LayerNorm -> qkv linear -> attention -> output linear + residual x, each stage
+    against the oracle on the GPU's own bf16 input to that stage."""
+    import vit_self_attention_b200 as vab
+    c = si.CONFIGS[cfg]
+    W = c.H * c.d
+    x = si.normal_bf16(700 + cfg, (c.B, c.N, W))
+    p = block_weights(W, 710 + cfg)
+    t = {k: dev(v) for k, v in p.items()}
+    xt = dev(x)
+    xn = vab.layernorm(xt, t["g"], t["be"], 1e-6)
+    qkv = vab.linear(xn, t["wqkv"], t["bqkv"])
+    o = vab.attention(qkv.view(c.B, c.N, 3, c.H, c.d), c.scale)
+    y = vab.linear(o.view(c.B, c.N, W), t["wo"], t["bo"], xt)
+    torch.cuda.synchronize()
+    assert_close_bf16(f64(xn), oracle.layernorm_bf16(x, p["g"], p["be"], 1e-6), "LayerNorm stage")
+    assert_close_bf16(f64(qkv), oracle.linear_bf16(host(xn), p["wqkv"], p["bqkv"]), "qkv stage")
+    assert_parity(f64(o), oracle.attention_packed_bf16(host(qkv).reshape(c.B, c.N, 3, c.H, c.d),
+                                                       c.scale), "attention stage")
+    ob = host(o).reshape(c.B, c.N, W)
+    assert_close_bf16(f64(y), oracle.linear_bf16(ob, p["wo"], p["bo"], x),
+                      "output projection + residual stage",
+                      mag=residual_magnitude(ob, p["wo"], p["bo"], x))
+
+
+def test_half_block_graph_capture():
+    """Two layers of the chain captured in one CUDA graph and replayed give the same bytes
+    as the eager calls."""
+    import vit_self_attention_b200 as vab
+    c = si.CONFIGS[1]
+    W = c.H * c.d
+    x0 = dev(si.normal_bf16(800, (c.B, c.N, W)))
+    layers = [{k: dev(v) for k, v in block_weights(W, 810 + 10 * i).items()} for i in range(2)]
+    ws = torch.empty(vab.vla_linear_workspace_bytes(), dtype=torch.uint8, device="cuda")
+    bufs = {"xn": torch.empty_like(x0), "qkv": torch.empty((c.B, c.N, 3 * W), dtype=torch.bfloat16,
+                                                            device="cuda"),
+            "o": torch.empty((c.B, c.N, c.H, c.d), dtype=torch.bfloat16, device="cuda")}
+
+    def run(x):
+        for p in layers:
+            vab.layernorm(x, p["g"], p["be"], 1e-6, out=bufs["xn"])
+            vab.linear(bufs["xn"], p["wqkv"], p["bqkv"], out=bufs["qkv"], workspace=ws)
+            vab.attention(bufs["qkv"].view(c.B, c.N, 3, c.H, c.d), c.scale, out=bufs["o"])
+            vab.linear(bufs["o"].view(c.B, c.N, W), p["wo"], p["bo"], x, out=x, workspace=ws)
+
+    eager = x0.clone()
+    run(eager)
+    torch.cuda.synchronize()
+    xg = x0.clone()
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        run(x0.clone())  # warm-up (plans, algorithms) outside the capture
+    torch.cuda.current_stream().wait_stream(side)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=side):
+        run(xg)
+    xg.copy_(x0)
+    g.replay()
+    torch.cuda.synchronize()
+    assert torch.equal(xg, eager)

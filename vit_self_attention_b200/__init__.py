@@ -46,6 +46,12 @@ _lib.vla_attn_set_wait_limit_ns.argtypes = [ctypes.c_uint64]
 _lib.vla_attn_set_wait_limit_ns.restype = None
 _lib.vla_attn_set_test_stall.argtypes = [_I]
 _lib.vla_attn_set_test_stall.restype = None
+_lib.vla_layernorm_fwd.argtypes = [_VP, _VP, _VP, _VP, _I, _I, ctypes.c_float, _VP]
+_lib.vla_layernorm_fwd.restype = _I
+_lib.vla_linear_fwd.argtypes = [_VP, _VP, _VP, _VP, _VP, _I, _I, _I, _VP, ctypes.c_size_t, _VP]
+_lib.vla_linear_fwd.restype = _I
+_lib.vla_linear_workspace_bytes.argtypes = []
+_lib.vla_linear_workspace_bytes.restype = ctypes.c_size_t
 
 # Status codes of include/vla_attn.h
 OK = 0
@@ -63,7 +69,7 @@ EXPORTED_SYMBOLS = (
     "vla_attn_fwd", "vla_attn_fwd_host", "vla_attn_strerror", "vla_attn_last_device_status",
     "vla_attn_reset_device_status", "vla_attn_max_tokens", "vla_attn_launch_count",
     "vla_attn_set_wait_limit_ns",
-    "vla_attn_set_test_stall",
+    "vla_attn_set_test_stall", "vla_layernorm_fwd", "vla_linear_fwd", "vla_linear_workspace_bytes",
 )
 
 
@@ -144,6 +150,56 @@ def vla_attn_set_test_stall(enable: bool) -> None:
     _lib.vla_attn_set_test_stall(1 if enable else 0)
 
 
+def vla_layernorm_fwd(x, gamma, beta, y, M: int, W: int, eps: float, stream=None,
+                      check: bool = True) -> int:
+    """Enqueue LayerNorm over the last dimension (see include/vla_attn.h)."""
+    st = _lib.vla_layernorm_fwd(_addr(x), _addr(gamma), _addr(beta), _addr(y), int(M), int(W),
+                                float(eps), _stream(stream))
+    if check and st != OK:
+        raise VlaAttnError(st)
+    return st
+
+
+def vla_linear_workspace_bytes() -> int:
+    return int(_lib.vla_linear_workspace_bytes())
+
+
+def vla_linear_fwd(x, w, bias, res, y, M: int, K: int, N: int, workspace=None,
+                   workspace_bytes: int = 0, stream=None, check: bool = True) -> int:
+    """Enqueue ``y = x @ w.T + bias (+ res)`` (see include/vla_attn.h)."""
+    st = _lib.vla_linear_fwd(_addr(x), _addr(w), _addr(bias), _addr(res), _addr(y), int(M),
+                             int(K), int(N), _addr(workspace), int(workspace_bytes),
+                             _stream(stream))
+    if check and st != OK:
+        raise VlaAttnError(st)
+    return st
+
+
+def layernorm(x, gamma, beta, eps: float = 1e-6, out=None, stream=None):
+    """LayerNorm of a contiguous bf16 CUDA tensor over its last dimension."""
+    import torch
+    if x.dtype != torch.bfloat16 or not x.is_cuda or not x.is_contiguous():
+        raise ValueError("x must be a contiguous bf16 CUDA tensor")
+    W = int(x.shape[-1])
+    if out is None:
+        out = torch.empty_like(x)
+    vla_layernorm_fwd(x, gamma, beta, out, x.numel() // W, W, eps, stream)
+    return out
+
+
+def linear(x, w, bias=None, res=None, out=None, workspace=None, stream=None):
+    """``x @ w.T + bias (+ res)`` for contiguous bf16 CUDA tensors (``w`` is ``[N, K]``)."""
+    import torch
+    N, K = (int(v) for v in w.shape)
+    M = x.numel() // K
+    if out is None:
+        out = torch.empty(tuple(x.shape[:-1]) + (N,), dtype=torch.bfloat16, device=x.device)
+    if workspace is None:
+        workspace = torch.empty(vla_linear_workspace_bytes(), dtype=torch.uint8, device=x.device)
+    vla_linear_fwd(x, w, bias, res, out, M, K, N, workspace, workspace.numel(), stream)
+    return out
+
+
 def attention(qkv, scale: float | None = None, out=None, stream=None):
     """Convenience wrapper for a contiguous bf16 CUDA tensor ``qkv`` of shape
     ``[B, N, 3, H, d]``; returns ``out`` (allocated by torch if None) ``[B, N, H, d]``."""
@@ -166,5 +222,7 @@ def attention(qkv, scale: float | None = None, out=None, stream=None):
 __all__ = [
     "LIBRARY_PATH", "EXPORTED_SYMBOLS", "VlaAttnError", "vla_attn_fwd", "vla_attn_fwd_host",
     "vla_attn_strerror", "vla_attn_last_device_status", "vla_attn_reset_device_status",
-    "vla_attn_max_tokens", "vla_attn_launch_count", "vla_attn_set_wait_limit_ns", "vla_attn_set_test_stall", "attention",
+    "vla_attn_max_tokens", "vla_attn_launch_count", "vla_attn_set_wait_limit_ns",
+    "vla_attn_set_test_stall", "vla_layernorm_fwd", "vla_linear_fwd", "vla_linear_workspace_bytes",
+    "layernorm", "linear", "attention",
 ]

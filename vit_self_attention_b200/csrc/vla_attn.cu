@@ -342,3 +342,7 @@ void vla_attn_set_wait_limit_ns(uint64_t ns) { g_wait_limit_ns.store(ns); }
 void vla_attn_set_test_stall(int enable) { g_test_stall.store(enable ? 1 : 0); }
 
 }  // extern "C"
+
+// LayerNorm and the linear layers around the attention core (same host
+// helpers: device and pointer-range checks, launch counter).
+#include "block_ops.cuh"
