@@ -181,6 +181,27 @@ int vla_linear_fwd(const void* x, const void* w, const void* bias, const void* r
 /* Recommended workspace size for vla_linear_fwd (bytes). */
 size_t vla_linear_workspace_bytes(void);
 
+/*
+ * vla_linear_fwd without a caller workspace and without any allocation: the
+ * cuBLASLt workspace is a file-scope device array of
+ * vla_linear_static_workspace_bytes() (8 MiB) per device, whose address is
+ * looked up once per device with cudaGetSymbolAddress.  cuBLASLt is asked
+ * only for algorithms that fit that array; a shape with none is rejected
+ * (VLA_ATTN_ERR_CUDA).  Arguments and results otherwise as vla_linear_fwd.
+ *   Calls that overlap on the GPU (on different streams, or from different
+ *   host threads without ordering) share the array and race; order them on
+ *   one stream.  The first call for a device and shape does the set-up (the
+ *   symbol lookup, the cuBLASLt handle and plan): make it before any stream
+ *   capture that records later calls.
+ * The pages have no counterpart of this entry point (a deployment variant of
+ * the linear layer, not a step of the method).
+ */
+int vla_linear_fwd_static(const void* x, const void* w, const void* bias, const void* res, void* y,
+                          int M, int K, int N, void* stream);
+
+/* Size of the fixed workspace of vla_linear_fwd_static (bytes). */
+size_t vla_linear_static_workspace_bytes(void);
+
 #ifdef __cplusplus
 }
 #endif

@@ -52,6 +52,10 @@ _lib.vla_linear_fwd.argtypes = [_VP, _VP, _VP, _VP, _VP, _I, _I, _I, _VP, ctypes
 _lib.vla_linear_fwd.restype = _I
 _lib.vla_linear_workspace_bytes.argtypes = []
 _lib.vla_linear_workspace_bytes.restype = ctypes.c_size_t
+_lib.vla_linear_fwd_static.argtypes = [_VP, _VP, _VP, _VP, _VP, _I, _I, _I, _VP]
+_lib.vla_linear_fwd_static.restype = _I
+_lib.vla_linear_static_workspace_bytes.argtypes = []
+_lib.vla_linear_static_workspace_bytes.restype = ctypes.c_size_t
 
 # Status codes of include/vla_attn.h
 OK = 0
@@ -70,6 +74,7 @@ EXPORTED_SYMBOLS = (
     "vla_attn_reset_device_status", "vla_attn_max_tokens", "vla_attn_launch_count",
     "vla_attn_set_wait_limit_ns",
     "vla_attn_set_test_stall", "vla_layernorm_fwd", "vla_linear_fwd", "vla_linear_workspace_bytes",
+    "vla_linear_fwd_static", "vla_linear_static_workspace_bytes",
 )
 
 
@@ -175,6 +180,21 @@ def vla_linear_fwd(x, w, bias, res, y, M: int, K: int, N: int, workspace=None,
     return st
 
 
+def vla_linear_static_workspace_bytes() -> int:
+    return int(_lib.vla_linear_static_workspace_bytes())
+
+
+def vla_linear_fwd_static(x, w, bias, res, y, M: int, K: int, N: int, stream=None,
+                          check: bool = True) -> int:
+    """``vla_linear_fwd`` with the library's fixed device workspace (no allocation;
+    overlapping calls race -- see the header)."""
+    st = _lib.vla_linear_fwd_static(_addr(x), _addr(w), _addr(bias), _addr(res), _addr(y),
+                                    int(M), int(K), int(N), _stream(stream))
+    if check and st != OK:
+        raise VlaAttnError(st)
+    return st
+
+
 def layernorm(x, gamma, beta, eps: float = 1e-6, out=None, stream=None):
     """LayerNorm of a contiguous bf16 CUDA tensor over its last dimension."""
     import torch
@@ -224,5 +244,6 @@ __all__ = [
     "vla_attn_strerror", "vla_attn_last_device_status", "vla_attn_reset_device_status",
     "vla_attn_max_tokens", "vla_attn_launch_count", "vla_attn_set_wait_limit_ns",
     "vla_attn_set_test_stall", "vla_layernorm_fwd", "vla_linear_fwd", "vla_linear_workspace_bytes",
-    "layernorm", "linear", "attention",
+    "vla_linear_fwd_static", "vla_linear_static_workspace_bytes", "layernorm", "linear",
+    "attention",
 ]

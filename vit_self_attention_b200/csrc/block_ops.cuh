@@ -198,6 +198,28 @@ int lt_plan(int dev, int M, int K, int N, bool bias, bool res, size_t ws, LtPlan
 
 constexpr size_t kLinearWorkspaceBytes = 32u << 20;
 
+// Fixed cuBLASLt workspace of vla_linear_fwd_static: one per device context.
+constexpr size_t kStaticWorkspaceBytes = 8u << 20;
+__device__ __align__(256) unsigned char g_static_workspace[kStaticWorkspaceBytes];
+
+std::mutex g_static_ws_mutex;
+void* g_static_ws_addr[kMaxDevices] = {};
+
+// Device address of this device's static workspace (looked up once per device).
+int static_workspace(int dev, void** out) {
+  std::lock_guard<std::mutex> lock(g_static_ws_mutex);
+  if (g_static_ws_addr[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_static_workspace) != cudaSuccess || p == nullptr) {
+      (void)cudaGetLastError();
+      return VLA_ATTN_ERR_CUDA;
+    }
+    g_static_ws_addr[dev] = p;
+  }
+  *out = g_static_ws_addr[dev];
+  return VLA_ATTN_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -240,6 +262,19 @@ int vla_layernorm_fwd(const void* x, const void* gamma, const void* beta, void* 
 }
 
 size_t vla_linear_workspace_bytes(void) { return kLinearWorkspaceBytes; }
+
+size_t vla_linear_static_workspace_bytes(void) { return kStaticWorkspaceBytes; }
+
+int vla_linear_fwd_static(const void* x, const void* w, const void* bias, const void* res, void* y,
+                          int M, int K, int N, void* stream) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return VLA_ATTN_ERR_CUDA;
+  if (dev < 0 || dev >= kMaxDevices) return VLA_ATTN_ERR_DEVICE;
+  void* ws = nullptr;
+  const int rc = static_workspace(dev, &ws);
+  if (rc != VLA_ATTN_OK) return rc;
+  return vla_linear_fwd(x, w, bias, res, y, M, K, N, ws, kStaticWorkspaceBytes, stream);
+}
 
 int vla_linear_fwd(const void* x, const void* w, const void* bias, const void* res, void* y,
                    int M, int K, int N, void* workspace, size_t workspace_bytes, void* stream) {
