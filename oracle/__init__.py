@@ -7,7 +7,8 @@ imports nothing from the CUDA package.
 
 The arithmetic lives in ``vla_attn_oracle.cpp`` (plain definitions of
 ``O = softmax(Q K^T * scale) V`` per image and head, of LayerNorm over the last
-dimension and of ``x @ w.T + bias (+ res)``, fp64 throughout); this
+dimension, of ``x @ w.T + bias (+ res)``, of the fused residual add + LayerNorm and
+of the linear layer with a GELU, fp64 throughout); this
 module only marshals numpy arrays through ctypes.  ``OracleLib`` can wrap any
 build of that source (the tests compile deliberately broken copies to show
 that the pins catch them); the module-level functions use the real build.
@@ -40,6 +41,13 @@ class OracleLib:
         lib.oracle_layernorm_bf16.restype = _I
         lib.oracle_linear_bf16.argtypes = [_U16P, _U16P, _U16P, _U16P, _DP, _I, _I, _I, _I]
         lib.oracle_linear_bf16.restype = _I
+        lib.oracle_round_bf16.argtypes = [_DP, _U16P, ctypes.c_long]
+        lib.oracle_round_bf16.restype = _I
+        lib.oracle_add_layernorm_bf16.argtypes = [_U16P, _U16P, _U16P, _U16P, _U16P, _DP, _I, _I,
+                                                  ctypes.c_double, _I]
+        lib.oracle_add_layernorm_bf16.restype = _I
+        lib.oracle_linear_gelu_bf16.argtypes = [_U16P, _U16P, _U16P, _DP, _I, _I, _I, _I]
+        lib.oracle_linear_gelu_bf16.restype = _I
         lib.oracle_attn_f64.argtypes = [_DP, _DP, _DP, _DP, _I, _I, _I, _I, ctypes.c_double, _I]
         lib.oracle_attn_f64.restype = _I
         lib.oracle_attn_probs_f64.argtypes = [_DP, _DP, _DP, _I, _I, _I, _I, ctypes.c_double]
@@ -153,6 +161,56 @@ class OracleLib:
             raise ValueError(f"oracle_linear_bf16 rejected the input (rc={rc})")
         return out
 
+    def round_bf16(self, v) -> np.ndarray:
+        """bf16 bits of finite fp64 values, rounded to nearest, ties to even."""
+        v = np.ascontiguousarray(v, dtype=np.float64)
+        out = np.empty(v.shape, dtype=np.uint16)
+        rc = self._lib.oracle_round_bf16(_ptr(v, ctypes.c_double), _ptr(out, ctypes.c_uint16),
+                                         int(v.size))
+        if rc != 0:
+            raise ValueError("oracle_round_bf16: non-finite input")
+        return out
+
+    def add_layernorm_bf16(self, x_bits, r_bits, gamma_bits, beta_bits, eps: float,
+                           threads: int = 0) -> tuple[np.ndarray, np.ndarray]:
+        """``(s, y)``: the residual stream ``s = bf16(x + r)`` (bits) and fp64
+        ``y = LayerNorm(s)`` over the last dimension."""
+        x = np.ascontiguousarray(x_bits, dtype=np.uint16)
+        r = np.ascontiguousarray(r_bits, dtype=np.uint16)
+        if r.shape != x.shape:
+            raise ValueError("x and r must have one shape")
+        W = int(x.shape[-1])
+        M = int(x.size // W)
+        g = np.ascontiguousarray(gamma_bits, dtype=np.uint16).reshape(W)
+        b = np.ascontiguousarray(beta_bits, dtype=np.uint16).reshape(W)
+        s = np.empty(x.shape, dtype=np.uint16)
+        y = np.empty(x.shape, dtype=np.float64)
+        rc = self._lib.oracle_add_layernorm_bf16(
+            _ptr(x, ctypes.c_uint16), _ptr(r, ctypes.c_uint16), _ptr(g, ctypes.c_uint16),
+            _ptr(b, ctypes.c_uint16), _ptr(s, ctypes.c_uint16), _ptr(y, ctypes.c_double), M, W,
+            float(eps), int(threads))
+        if rc != 0:
+            raise ValueError(f"oracle_add_layernorm_bf16 rejected the input (rc={rc})")
+        return s, y
+
+    def linear_gelu_bf16(self, x_bits, w_bits, bias_bits=None, threads: int = 0) -> np.ndarray:
+        """fp64 ``gelu(x @ w.T + bias)`` (tanh form) for bf16 ``x [..., K]``, ``w [N, K]``."""
+        x = np.ascontiguousarray(x_bits, dtype=np.uint16)
+        w = np.ascontiguousarray(w_bits, dtype=np.uint16)
+        N, K = (int(v) for v in w.shape)
+        if x.shape[-1] != K:
+            raise ValueError("x and w disagree on K")
+        M = int(x.size // K)
+        b = None if bias_bits is None else np.ascontiguousarray(bias_bits, dtype=np.uint16).reshape(N)
+        out = np.empty(x.shape[:-1] + (N,), dtype=np.float64)
+        rc = self._lib.oracle_linear_gelu_bf16(
+            _ptr(x, ctypes.c_uint16), _ptr(w, ctypes.c_uint16),
+            None if b is None else _ptr(b, ctypes.c_uint16), _ptr(out, ctypes.c_double),
+            M, K, N, int(threads))
+        if rc != 0:
+            raise ValueError(f"oracle_linear_gelu_bf16 rejected the input (rc={rc})")
+        return out
+
 
 _default: OracleLib | None = None
 
@@ -193,8 +251,21 @@ def linear_bf16(x_bits, w_bits, bias_bits=None, res_bits=None, threads: int = 0)
     return lib().linear_bf16(x_bits, w_bits, bias_bits, res_bits, threads)
 
 
+def round_bf16(v) -> np.ndarray:
+    return lib().round_bf16(v)
+
+
+def add_layernorm_bf16(x_bits, r_bits, gamma_bits, beta_bits, eps: float, threads: int = 0):
+    return lib().add_layernorm_bf16(x_bits, r_bits, gamma_bits, beta_bits, eps, threads)
+
+
+def linear_gelu_bf16(x_bits, w_bits, bias_bits=None, threads: int = 0) -> np.ndarray:
+    return lib().linear_gelu_bf16(x_bits, w_bits, bias_bits, threads)
+
+
 SOURCE = _build.SRC
 
 __all__ = ["OracleLib", "lib", "attention_f64", "probs_f64", "attention_packed_bf16",
-           "attention_rows_packed_bf16", "layernorm_bf16", "linear_bf16", "default_threads",
+           "attention_rows_packed_bf16", "layernorm_bf16", "linear_bf16", "round_bf16",
+           "add_layernorm_bf16", "linear_gelu_bf16", "default_threads",
            "SOURCE"]

@@ -291,3 +291,81 @@ int oracle_linear_bf16(const uint16_t* x, const uint16_t* w, const uint16_t* bia
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// The rest of a ViT encoder layer, same plain fp64 style:
+//
+//   Residual add + LayerNorm (one fused operator on the FluxVLA page, Triton
+//   fused kernels: norm fusion).  The sum is the residual stream, which is
+//   stored in bf16, and the LayerNorm reads that stored stream:
+//     s[m,i] = bf16_rne(x[m,i] + r[m,i])       (returned as bf16 bits)
+//     y[m,i] = LayerNorm(s)[m,i]               (as above, fp64)
+//   The fusion must give what the two separate steps give, so s is rounded
+//   exactly as an unfused add that stores bf16 would round it.
+//
+//   Linear layer + bias + GELU (same page, same section: matrix multiply with
+//   bias and activation fused after the tiled product), the first MLP layer:
+//     a[m,n] = sum_k x[m,k] * w[n,k] + bias[n]
+//     y[m,n] = a/2 * (1 + tanh(sqrt(2/pi) * (a + 0.044715 a^3)))
+//   The pages do not say which GELU; this is the tanh form of Hendrycks and
+//   Gimpel's paper, the one SigLIP (the Pi0 vision encoder) uses.
+
+namespace {
+
+// Round-to-nearest-even of a finite double to bf16 (8 significant bits,
+// 8 exponent bits), returned as bits.  From the format's definition: the
+// value is scaled so that its quantum becomes 1, rounded to an integer with
+// ties to even (the default floating-point rounding mode), and scaled back.
+uint16_t round_bf16(double v) {
+  if (v == 0.0) return std::signbit(v) ? 0x8000u : 0u;
+  int e = 0;
+  (void)std::frexp(v, &e);                     // |v| = f 2^e, f in [0.5, 1)
+  const int q = std::max(e - 8, -133);         // quantum 2^q; subnormals share 2^-133
+  const double r = std::ldexp(std::nearbyint(std::ldexp(v, -q)), q);
+  if (std::fabs(r) >= std::ldexp(1.0, 128)) return std::signbit(v) ? 0xFF80u : 0x7F80u;
+  const float f = static_cast<float>(r);       // exact: r has at most 8 significant bits
+  uint32_t u;
+  std::memcpy(&u, &f, sizeof(u));
+  return static_cast<uint16_t>(u >> 16);
+}
+
+}  // namespace
+
+extern "C" {
+
+int oracle_round_bf16(const double* v, uint16_t* bits, long n) {
+  for (long i = 0; i < n; ++i) {
+    if (!std::isfinite(v[i])) return -1;
+    bits[i] = round_bf16(v[i]);
+  }
+  return 0;
+}
+
+// s = bf16(x + r) (bits), y = LayerNorm(s) (fp64); M rows of width W.
+int oracle_add_layernorm_bf16(const uint16_t* x, const uint16_t* r, const uint16_t* gamma,
+                              const uint16_t* beta, uint16_t* s, double* y, int M, int W,
+                              double eps, int nthreads) {
+  if (M < 0 || W <= 0 || !(eps >= 0.0)) return -1;
+  parallel_for(static_cast<long>(M), nthreads, [&](long m) {
+    const std::ptrdiff_t off = m * static_cast<std::ptrdiff_t>(W);
+    for (int i = 0; i < W; ++i)
+      s[off + i] = round_bf16(widen_bf16(x[off + i]) + widen_bf16(r[off + i]));
+  });
+  return oracle_layernorm_bf16(s, gamma, beta, y, M, W, eps, nthreads);
+}
+
+// y[m,n] = gelu(sum_k x[m,k] w[n,k] + bias[n])  (bf16 inputs, fp64 y; bias may be null).
+int oracle_linear_gelu_bf16(const uint16_t* x, const uint16_t* w, const uint16_t* bias,
+                            double* y, int M, int K, int N, int nthreads) {
+  const int rc = oracle_linear_bf16(x, w, bias, nullptr, y, M, K, N, nthreads);
+  if (rc != 0) return rc;
+  const double c = std::sqrt(2.0 / 3.14159265358979323846);
+  const long n = static_cast<long>(M) * N;
+  for (long i = 0; i < n; ++i) {
+    const double a = y[i];
+    y[i] = 0.5 * a * (1.0 + std::tanh(c * (a + 0.044715 * a * a * a)));
+  }
+  return 0;
+}
+
+}  // extern "C"

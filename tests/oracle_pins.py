@@ -391,6 +391,121 @@ def pin_linear_brute_force_and_torch(lib):
     _close(lib.linear_bf16(x, w, b), want, 1e-10, "torch addmm fp64")
 
 
+# ------------------------------------------------------------ bf16 rounding
+# Round to nearest, ties to even, of the residual stream's sum (the fused residual
+# add + LayerNorm stores s = x + r in bf16).
+
+def pin_round_bf16_ties_and_torch(lib):
+    """Hand-worked ties and edges, then torch's float32 -> bfloat16 conversion (round to
+    nearest even) on random float32 values, subnormals and ties included."""
+    import torch
+    cases = [(1.0, 0x3F80), (1.0 + 2.0 ** -8, 0x3F80),           # tie -> even (down)
+             (1.0 + 3 * 2.0 ** -8, 0x3F82),                         # tie -> even (up)
+             (1.0 + 2.0 ** -8 + 2.0 ** -30, 0x3F81),                # just above a tie
+             (-3.0, 0xC040), (0.0, 0x0000), (-0.0, 0x8000),
+             (2.0 ** -133, 0x0001), (1.5 * 2.0 ** -133, 0x0002),    # subnormal tie -> even
+             (2.0 ** -134, 0x0000),                                 # subnormal tie -> zero
+             (255.5 * 2.0 ** 120, 0x7F80), (255.25 * 2.0 ** 120, 0x7F7F)]
+    got = lib.round_bf16(np.array([v for v, _ in cases]))
+    for (v, want), g in zip(cases, got):
+        assert int(g) == want, f"round_bf16({v!r}) = {int(g):#06x}, want {want:#06x}"
+    rng = _rng(40)
+    v = rng.normal(size=4000).astype(np.float32) * np.float32(3.0)
+    ties = (_bf16(rng.normal(size=500)).astype(np.uint32) << 16) | np.uint32(0x8000)
+    tiny = rng.normal(size=500).astype(np.float32) * np.float32(1e-39)
+    v = np.concatenate([v, ties.view(np.float32), tiny])
+    want = torch.from_numpy(v).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    got = lib.round_bf16(v.astype(np.float64))
+    assert np.array_equal(got, want), f"{int((got != want).sum())} roundings differ from torch"
+
+
+# ------------------------------------------------- residual add + LayerNorm
+# s = bf16(x + r), y = LayerNorm(s)  ("FluxVLA docs, inference acceleration", Triton
+# fused kernels: residual add + LayerNorm in one kernel).
+
+def pin_add_layernorm_reductions(lib):
+    """r = 0 gives s = x and y = LayerNorm(x); sums that bf16 holds exactly are exact;
+    the add is symmetric; torch's bf16 add gives the same stream bits."""
+    import torch
+    W = 48
+    x = _bf16(_rng(41).normal(size=(5, W)))
+    g = _bf16(_rng(42).normal(1.0, 0.3, size=W))
+    b = _bf16(_rng(43).normal(0.0, 0.3, size=W))
+    s, y = lib.add_layernorm_bf16(x, _bits(np.zeros((5, W))), g, b, 1e-6)
+    assert np.array_equal(s, x), "r = 0 must leave the stream unchanged"
+    _close(y, lib.layernorm_bf16(x, g, b, 1e-6), 0.0, "r = 0 reduces to LayerNorm")
+    xi = _rng(44).integers(-60, 60, size=(3, W)).astype(np.float64)
+    ri = _rng(45).integers(-60, 60, size=(3, W)).astype(np.float64)
+    s, _ = lib.add_layernorm_bf16(_bits(xi), _bits(ri), g, b, 1e-6)
+    assert np.array_equal(s, _bits(xi + ri)), "exact integer sums"
+    r = _bf16(_rng(46).normal(0.0, 4.0, size=(5, W)))
+    s1, y1 = lib.add_layernorm_bf16(x, r, g, b, 1e-5)
+    s2, y2 = lib.add_layernorm_bf16(r, x, g, b, 1e-5)
+    assert np.array_equal(s1, s2)
+    _close(y1, y2, 0.0, "symmetric add")
+    tx = torch.from_numpy(x.view(np.int16)).view(torch.bfloat16)
+    tr = torch.from_numpy(r.view(np.int16)).view(torch.bfloat16)
+    want = (tx + tr).view(torch.int16).numpy().view(np.uint16)
+    assert np.array_equal(s1, want), "stream bits differ from torch's bf16 add"
+
+
+def pin_add_layernorm_torch(lib):
+    """torch: the bf16 residual add, then fp64 layer_norm of the stored stream, at the
+    ViT-L width."""
+    import torch
+    M, W = 30, 1024
+    x = _bf16(_rng(47).normal(0.2, 1.5, size=(M, W)))
+    r = _bf16(_rng(48).normal(-0.1, 0.8, size=(M, W)))
+    g = _bf16(_rng(49).normal(1.0, 0.2, size=W))
+    b = _bf16(_rng(50).normal(0.0, 0.2, size=W))
+    tb = lambda t: torch.from_numpy(t.view(np.int16)).view(torch.bfloat16)
+    stream = (tb(x) + tb(r)).double()
+    want = torch.nn.functional.layer_norm(stream, (W,), tb(g).double(), tb(b).double(), 1e-6)
+    s, y = lib.add_layernorm_bf16(x, r, g, b, 1e-6)
+    _close(y, want.numpy(), 1e-10, "torch add + layer_norm fp64")
+
+
+# --------------------------------------------------------- linear + GELU
+# y = gelu(x @ w.T + bias), tanh form (same page, same section: matrix multiply with
+# bias and activation fused).
+
+def pin_linear_gelu_torch_and_erf(lib):
+    """torch's fp64 tanh GELU after addmm; within the tanh form's published gap
+    (< 5e-4) of the exact x Phi(x), and measurably not the exact form."""
+    import torch
+    from scipy.special import erf
+    M, K, N = 40, 1152, 512
+    x = _bf16(_rng(51).normal(size=(M, K)))
+    w = _bf16(_rng(52).normal(size=(N, K)) * 2.0 / math.sqrt(K))
+    b = _bf16(_rng(53).normal(size=N))
+    tw = lambda t: torch.from_numpy(si.bf16_bits_to_f32(t).astype(np.float64))
+    pre = torch.addmm(tw(b), tw(x), tw(w).T)
+    want = torch.nn.functional.gelu(pre, approximate="tanh").numpy()
+    got = lib.linear_gelu_bf16(x, w, b)
+    _close(got, want, 1e-12, "torch gelu(tanh) fp64")
+    a = pre.numpy()
+    exact = 0.5 * a * (1.0 + erf(a / math.sqrt(2.0)))
+    gap = np.abs(got - exact).max()
+    assert gap < 5e-4, f"tanh GELU {gap} away from the exact form"
+    assert gap > 1e-4, "this is the exact (erf) GELU, not the tanh form"
+
+
+def pin_linear_gelu_closed_forms(lib):
+    """gelu(0) = 0; gelu(a) = a for large a and 0 for large -a; gelu(a) - gelu(-a) = a
+    (odd part of the tanh form), checked through weights w and -w."""
+    K = 16
+    x = _bf16(_rng(54).normal(size=(4, K)))
+    zero_w = _bits(np.zeros((8, K)))
+    _close(lib.linear_gelu_bf16(x, zero_w), np.zeros((4, 8)), 0.0, "gelu(0)")
+    big = _bits(np.array([10.0, -10.0, 24.0, -24.0, 0.0, 0.0, 0.0, 0.0]))
+    y = lib.linear_gelu_bf16(x, zero_w, big)
+    _close(y[:, :4], np.broadcast_to([10.0, 0.0, 24.0, 0.0], (4, 4)), 1e-12, "saturation")
+    w = _bf16(_rng(55).normal(size=(8, K)))
+    minus_w = w ^ np.uint16(0x8000)
+    diff = lib.linear_gelu_bf16(x, w) - lib.linear_gelu_bf16(x, minus_w)
+    _close(diff, lib.linear_bf16(x, w), 1e-12, "odd part")
+
+
 ALL_PINS = [
     pin_golden_closed_forms,
     pin_single_token,
@@ -411,4 +526,9 @@ ALL_PINS = [
     pin_linear_closed_forms,
     pin_linear_permutation_and_linearity,
     pin_linear_brute_force_and_torch,
+    pin_round_bf16_ties_and_torch,
+    pin_add_layernorm_reductions,
+    pin_add_layernorm_torch,
+    pin_linear_gelu_torch_and_erf,
+    pin_linear_gelu_closed_forms,
 ]

@@ -52,6 +52,26 @@ MUTANTS = [
      "for (int k = 0; k < K - 1; ++k) acc += xm[k] * widen_bf16(wn[k]);"),
     ("linear_residual_dropped",
      "if (res != nullptr) acc += widen_bf16(res[m * static_cast<std::ptrdiff_t>(N) + n]);", ""),
+    ("round_toward_zero", "std::nearbyint(std::ldexp(v, -q))", "std::trunc(std::ldexp(v, -q))"),
+    ("round_ties_away", "std::nearbyint(std::ldexp(v, -q))", "std::round(std::ldexp(v, -q))"),
+    ("round_seven_bits", "const int q = std::max(e - 8, -133);",
+     "const int q = std::max(e - 7, -133);"),
+    ("round_subnormals_flushed", "const int q = std::max(e - 8, -133);",
+     "const int q = std::max(e - 8, -126);"),
+    ("add_ln_residual_dropped",
+     "s[off + i] = round_bf16(widen_bf16(x[off + i]) + widen_bf16(r[off + i]));",
+     "s[off + i] = round_bf16(widen_bf16(x[off + i]));"),
+    ("add_ln_normalises_x_not_stream",
+     "return oracle_layernorm_bf16(s, gamma, beta, y, M, W, eps, nthreads);",
+     "return oracle_layernorm_bf16(x, gamma, beta, y, M, W, eps, nthreads);"),
+    ("gelu_cubic_sign", "a + 0.044715 * a * a * a", "a - 0.044715 * a * a * a"),
+    ("gelu_half_dropped", "y[i] = 0.5 * a * (1.0 + std::tanh(", "y[i] = a * (1.0 + std::tanh("),
+    ("gelu_sqrt_two_over_pi_wrong", "std::sqrt(2.0 / 3.14159265358979323846)",
+     "std::sqrt(1.0 / 3.14159265358979323846)"),
+    ("gelu_bias_ignored", "oracle_linear_bf16(x, w, bias, nullptr, y, M, K, N, nthreads)",
+     "oracle_linear_bf16(x, w, nullptr, nullptr, y, M, K, N, nthreads)"),
+    ("gelu_is_sigmoid_form", "std::tanh(c * (a + 0.044715 * a * a * a))",
+     "std::tanh(0.851 * a)"),
 ]
 
 
