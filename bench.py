@@ -520,10 +520,13 @@ def _graph_time_us(fn, reps: int = 20, iters: int = 10) -> list[float]:
 
 
 def run_block(args) -> None:
-    """LayerNorm and the linear layers (qkv projection; output projection with the
-    residual add) on the encoder shapes and the bench batch, and the attention half of
-    a ViT block (LayerNorm -> qkv -> attention -> output projection + residual): one
-    layer at the bench batch, and the L-layer sequence for the encoder workloads."""
+    """The layers around the attention core on the encoder shapes and the bench batch:
+    LayerNorm, the fused residual add + LayerNorm, the qkv linear, the output projection
+    with the residual add, the MLP's fc1 + GELU and fc2 + residual; the attention half of
+    a ViT block and the whole pre-norm encoder layer (LN1 -> qkv -> attention -> output
+    projection + residual -> LN2 -> fc1 + GELU -> fc2 + residual), one layer at the bench
+    batch, and for the encoder workloads their L layers (fresh weights and activations per
+    layer) in one CUDA graph."""
     import math as _m
 
     import torch
@@ -536,70 +539,97 @@ def run_block(args) -> None:
     p_bf16 = float(peaks["bf16_tflops"]) * 1e12
     hbm = float(peaks["hbm_gbs"]) * 1e9
     ws = torch.empty(vab.vla_linear_workspace_bytes(), dtype=torch.uint8, device=dev)
+    mlp_width = {768: 3072, 1024: 4096, 1152: 4304}
 
     def t_(shape, mean=0.0, std=1.0, seed=1):
         b = si.normal_bf16(seed, shape, mean, std)
         return torch.from_numpy(b.view(np.int16)).to(dev).view(torch.bfloat16)
 
+    def layer_weights(W, F, seed):
+        return {"g": t_((W,), 1.0, 0.1, seed), "be": t_((W,), 0.0, 0.1, seed + 1),
+                "wq": t_((3 * W, W), 0.0, 1.0 / _m.sqrt(W), seed + 2),
+                "bq": t_((3 * W,), 0.0, 0.1, seed + 3),
+                "wo": t_((W, W), 0.0, 1.0 / _m.sqrt(W), seed + 4), "bo": t_((W,), 0.0, 0.1, seed + 5),
+                "g2": t_((W,), 1.0, 0.1, seed + 6), "be2": t_((W,), 0.0, 0.1, seed + 7),
+                "w1": t_((F, W), 0.0, 1.0 / _m.sqrt(W), seed + 8), "b1": t_((F,), 0.0, 0.1, seed + 9),
+                "w2": t_((W, F), 0.0, 1.0 / _m.sqrt(F), seed + 10), "b2": t_((W,), 0.0, 0.1, seed + 11)}
+
     for c in list(si.CONFIGS[1:4]) + [si.CONFIGS[4]]:
         W = c.H * c.d
+        F = mlp_width[W]
         M = c.B * c.N
         x = t_((c.B, c.N, W), 0.0, 1.0, 11)
-        g, be = t_((W,), 1.0, 0.1, 12), t_((W,), 0.0, 0.1, 13)
-        wq, bq = t_((3 * W, W), 0.0, 1.0 / _m.sqrt(W), 14), t_((3 * W,), 0.0, 0.1, 15)
-        wo, bo = t_((W, W), 0.0, 1.0 / _m.sqrt(W), 16), t_((W,), 0.0, 0.1, 17)
+        p = layer_weights(W, F, 12)
         xn = torch.empty_like(x)
         qkv = torch.empty((c.B, c.N, 3 * W), dtype=torch.bfloat16, device=dev)
         o = torch.empty((c.B, c.N, c.H, c.d), dtype=torch.bfloat16, device=dev)
         y = torch.empty_like(x)
-        ln = lambda: vab.layernorm(x, g, be, 1e-6, out=xn)
-        lq = lambda: vab.linear(xn, wq, bq, out=qkv, workspace=ws)
+        s2 = torch.empty_like(x)
+        a = torch.empty((c.B, c.N, F), dtype=torch.bfloat16, device=dev)
+        y2 = torch.empty_like(x)
+        ln = lambda: vab.layernorm(x, p["g"], p["be"], 1e-6, out=xn)
+        lq = lambda: vab.linear(xn, p["wq"], p["bq"], out=qkv, workspace=ws)
         at = lambda: vab.attention(qkv.view(c.B, c.N, 3, c.H, c.d), c.scale, out=o)
-        lo = lambda: vab.linear(o.view(c.B, c.N, W), wo, bo, x, out=y, workspace=ws)
-        ref = lambda: torch.addmm(bq, xn.view(M, W), wq.t(), out=qkv.view(M, 3 * W))
+        lo = lambda: vab.linear(o.view(c.B, c.N, W), p["wo"], p["bo"], x, out=y, workspace=ws)
+        ln2 = lambda: vab.layernorm(y, p["g2"], p["be2"], 1e-6, out=xn)
+        f1 = lambda: vab.linear_gelu(xn, p["w1"], p["b1"], out=a, workspace=ws)
+        f2 = lambda: vab.linear(a, p["w2"], p["b2"], y, out=y2, workspace=ws)
+        aln = lambda: vab.add_layernorm(x, y, p["g2"], p["be2"], 1e-6, out_s=s2, out_y=xn)
+        ref = lambda: torch.addmm(p["bq"], xn.view(M, W), p["wq"].t(), out=qkv.view(M, 3 * W))
         big = c.B * c.N >= 100000
         reps, iters = (3, 5) if big else (20, 10)
         med = lambda f: statistics.median(_graph_time_us(f, reps, iters))
         t_ln, t_q, t_at, t_o, t_ref = med(ln), med(lq), med(at), med(lo), med(ref)
-        fq, fo = 2.0 * M * W * 3 * W, 2.0 * M * W * W
-        rec = {"mode": "block", "workload": c.name, "tokens": M, "width": W,
+        t_f1, t_f2, t_aln = med(f1), med(f2), med(aln)
+        fq, fo, ff = 2.0 * M * W * 3 * W, 2.0 * M * W * W, 2.0 * M * W * F
+        rec = {"mode": "block", "workload": c.name, "tokens": M, "width": W, "mlp_width": F,
                "layernorm": {"us": t_ln, "gbs": 4.0 * M * W / t_ln / 1e3,
                              "frac_hbm": 4.0 * M * W / t_ln / 1e-6 / hbm},
+               "add_layernorm": {"us": t_aln, "gbs": 8.0 * M * W / t_aln / 1e3,
+                                 "frac_hbm": 8.0 * M * W / t_aln / 1e-6 / hbm},
                "qkv_linear": {"us": t_q, "tflops": fq / t_q / 1e6,
                               "frac_bf16": fq / t_q / 1e-6 / p_bf16,
                               "torch_addmm_us": t_ref},
                "attention": {"us": t_at, "tflops": c.flops() / t_at / 1e6},
                "out_linear_residual": {"us": t_o, "tflops": fo / t_o / 1e6,
-                                       "frac_bf16": fo / t_o / 1e-6 / p_bf16}}
-        chain = lambda: (ln(), lq(), at(), lo())
-        t_chain = med(chain)
-        rec["half_block_us"] = t_chain
-        rec["half_block_tflops"] = (fq + fo + c.flops()) / t_chain / 1e6
+                                       "frac_bf16": fo / t_o / 1e-6 / p_bf16},
+               "fc1_gelu": {"us": t_f1, "tflops": ff / t_f1 / 1e6,
+                            "frac_bf16": ff / t_f1 / 1e-6 / p_bf16},
+               "fc2_residual": {"us": t_f2, "tflops": ff / t_f2 / 1e6,
+                                "frac_bf16": ff / t_f2 / 1e-6 / p_bf16}}
+        t_half = med(lambda: (ln(), lq(), at(), lo()))
+        rec["half_block_us"] = t_half
+        rec["half_block_tflops"] = (fq + fo + c.flops()) / t_half / 1e6
+        layer_flops = fq + fo + 2.0 * ff + c.flops()
+        t_layer = med(lambda: (ln(), lq(), at(), lo(), ln2(), f1(), f2()))
+        rec["layer_us"] = t_layer
+        rec["layer_tflops"] = layer_flops / t_layer / 1e6
         if not big:
-            # The encoder's L layers (fresh weights and activations per layer) in one graph.
-            layers = []
-            for i in range(c.layers):
-                layers.append((t_((W,), 1.0, 0.1, 100 + 7 * i), t_((W,), 0.0, 0.1, 101 + 7 * i),
-                               t_((3 * W, W), 0.0, 1.0 / _m.sqrt(W), 102 + 7 * i),
-                               t_((3 * W,), 0.0, 0.1, 103 + 7 * i),
-                               t_((W, W), 0.0, 1.0 / _m.sqrt(W), 104 + 7 * i),
-                               t_((W,), 0.0, 0.1, 105 + 7 * i)))
-            xs = [x.clone() for _ in range(c.layers + 1)]
+            # The encoder's L whole layers (fresh weights and activations per layer) in one
+            # graph; the residual stream moves to a new buffer at every residual add.
+            layers = [layer_weights(W, F, 100 + 13 * i) for i in range(c.layers)]
+            xs = [x.clone() for _ in range(2 * c.layers + 1)]
 
             def encoder():
-                for i, (g_, b_, wq_, bq_, wo_, bo_) in enumerate(layers):
-                    vab.layernorm(xs[i], g_, b_, 1e-6, out=xn)
-                    vab.linear(xn, wq_, bq_, out=qkv, workspace=ws)
+                for i, q in enumerate(layers):
+                    h_in, h_mid, h_out = xs[2 * i], xs[2 * i + 1], xs[2 * i + 2]
+                    vab.layernorm(h_in, q["g"], q["be"], 1e-6, out=xn)
+                    vab.linear(xn, q["wq"], q["bq"], out=qkv, workspace=ws)
                     vab.attention(qkv.view(c.B, c.N, 3, c.H, c.d), c.scale, out=o)
-                    vab.linear(o.view(c.B, c.N, W), wo_, bo_, xs[i], out=xs[i + 1], workspace=ws)
+                    vab.linear(o.view(c.B, c.N, W), q["wo"], q["bo"], h_in, out=h_mid,
+                               workspace=ws)
+                    vab.layernorm(h_mid, q["g2"], q["be2"], 1e-6, out=xn)
+                    vab.linear_gelu(xn, q["w1"], q["b1"], out=a, workspace=ws)
+                    vab.linear(a, q["w2"], q["b2"], h_mid, out=h_out, workspace=ws)
 
             t_enc = statistics.median(_graph_time_us(encoder, 1, 20))
             rec["encoder_layers"] = c.layers
-            rec["encoder_half_blocks_us"] = t_enc
+            rec["encoder_us"] = t_enc
+            rec["encoder_tflops"] = c.layers * layer_flops / t_enc / 1e6
             rec["encoder_images_per_s"] = c.B / (t_enc * 1e-6)
             del layers, xs
         print(json.dumps(rec), flush=True)
-        del x, xn, qkv, o, y, wq, wo
+        del x, xn, qkv, o, y, s2, a, y2, p
         torch.cuda.empty_cache()
 
 
@@ -618,7 +648,7 @@ def main() -> None:
     ap.add_argument("--configs", action="store_true",
                     help="per-config report instead of the benchmark line (1 GPU)")
     ap.add_argument("--block", action="store_true",
-                    help="LayerNorm / linear layers and the attention half-block (1 GPU)")
+                    help="the layers around attention, whole encoder layers and encoders (1 GPU)")
     args = ap.parse_args()
     if args.configs:
         run_configs(args)

@@ -178,6 +178,35 @@ int vla_layernorm_fwd(const void* x, const void* gamma, const void* beta, void* 
 int vla_linear_fwd(const void* x, const void* w, const void* bias, const void* res, void* y,
                    int M, int K, int N, void* workspace, size_t workspace_bytes, void* stream);
 
+/*
+ * Residual add fused with LayerNorm ("FluxVLA docs, inference acceleration",
+ * Triton fused kernels, norm fusion: residual add + LayerNorm in one kernel):
+ *   s[m,i] = bf16(x[m,i] + r[m,i])      (sum in fp32, rounded to nearest even)
+ *   y[m,i] = LayerNorm(s)[m,i]          (as vla_layernorm_fwd, on the stored s)
+ * s is the new residual stream; normalising the stored bf16 values makes the
+ * result identical to a separate add followed by vla_layernorm_fwd.
+ *   x, r, s, y: [M, W] row-major bf16 device buffers; gamma, beta: [W] bf16.
+ *   Each output may be exactly x or r (in-place stream update) or disjoint
+ *   from them; s and y are disjoint; gamma and beta do not overlap an output.
+ *   Shapes, alignment, eps and errors as vla_layernorm_fwd.  One launch on
+ *   `stream`, no allocation, graph-capturable.
+ */
+int vla_add_layernorm_fwd(const void* x, const void* r, const void* gamma, const void* beta,
+                          void* s, void* y, int M, int W, float eps, void* stream);
+
+/*
+ * Linear layer with bias and GELU in one cuBLASLt matmul, the first layer of
+ * the ViT MLP (same page, Triton fused kernels: matrix multiply + bias +
+ * activation; the activation is GELU in its tanh form,
+ * a/2 (1 + tanh(sqrt(2/pi) (a + 0.044715 a^3))), as in SigLIP):
+ *   y[m,n] = gelu(sum_k x[m,k] * w[n,k] + bias[n])
+ *   Layout, alignment, workspace, bias (may be NULL), errors and the
+ *   fp32-accumulate, bf16-output arithmetic as vla_linear_fwd; there is no
+ *   residual input.  y must not overlap x, w, bias or the workspace.
+ */
+int vla_linear_gelu_fwd(const void* x, const void* w, const void* bias, void* y, int M, int K,
+                        int N, void* workspace, size_t workspace_bytes, void* stream);
+
 /* Recommended workspace size for vla_linear_fwd (bytes). */
 size_t vla_linear_workspace_bytes(void);
 

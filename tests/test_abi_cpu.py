@@ -146,3 +146,33 @@ def test_layernorm_and_linear_validation_on_host():
     assert lin(bias=BI + 2) == vab.ERR_ALIGN and lin(res=R + 4) == vab.ERR_ALIGN
     assert lin(ws=WS + 8) == vab.ERR_ALIGN
     assert vab.vla_linear_workspace_bytes() >= 1 << 20
+
+
+def test_add_layernorm_and_linear_gelu_validation_on_host():
+    """The fused residual add + LayerNorm and the linear + GELU entry points reject bad
+    arguments before touching a GPU."""
+    import math as _m
+
+    import vit_self_attention_b200 as vab
+    X, R, G, B_, S, Y = (0x10000000 + i * 0x1000000 for i in range(6))
+
+    def aln(x=X, r=R, g=G, b=B_, s=S, y=Y, M=4, W=1024, eps=1e-6):
+        return vab.vla_add_layernorm_fwd(x, r, g, b, s, y, M, W, eps, stream=0, check=False)
+
+    for kw in ("x", "r", "g", "b", "s", "y"):
+        assert aln(**{kw: None}) == vab.ERR_NULL, kw
+    assert aln(M=0) == vab.ERR_SHAPE and aln(W=-8) == vab.ERR_SHAPE
+    assert aln(W=20) == vab.ERR_UNSUPPORTED and aln(W=4096) == vab.ERR_UNSUPPORTED
+    assert aln(eps=-1e-6) == vab.ERR_SCALE and aln(eps=_m.inf) == vab.ERR_SCALE
+    assert aln(r=R + 2) == vab.ERR_ALIGN and aln(s=S + 8) == vab.ERR_ALIGN
+
+    W_, BI, WS = 0x17000000, 0x18000000, 0x19000000
+
+    def lg(x=X, w=W_, bias=BI, y=Y, M=4, K=1152, N=4304, ws=WS, wsb=1 << 20):
+        return vab.vla_linear_gelu_fwd(x, w, bias, y, M, K, N, ws, wsb, stream=0, check=False)
+
+    assert lg(x=None) == vab.ERR_NULL and lg(w=None) == vab.ERR_NULL and lg(y=None) == vab.ERR_NULL
+    assert lg(ws=None) == vab.ERR_NULL
+    assert lg(M=0) == vab.ERR_SHAPE and lg(N=-8) == vab.ERR_SHAPE
+    assert lg(K=12) == vab.ERR_UNSUPPORTED and lg(N=4302) == vab.ERR_UNSUPPORTED
+    assert lg(bias=BI + 2) == vab.ERR_ALIGN and lg(y=Y + 4) == vab.ERR_ALIGN

@@ -1,4 +1,5 @@
-"""LayerNorm and linear layers around the attention core vs. the fp64 oracle.
+"""LayerNorm, residual add + LayerNorm, linear and linear + GELU layers around the
+attention core vs. the fp64 oracle, and whole encoder layers stage by stage.
 
 Stage-wise: every GPU stage is compared with the oracle on identical bf16 inputs
 (the GPU's own bf16 output of the previous stage feeds the oracle's next stage).
@@ -7,7 +8,11 @@ mean |err| <= 2e-3); LayerNorm and linear outputs use the bound derived from the
 arithmetic (bf16 rounding of an fp32 result, possibly twice -- GEMM + bias, then the
 residual sum -- each at most 2^-9 of what it rounds: elementwise
 |err| <= 2^-7 (|x w^T + b| + |res|) + 2^-9, mean error <= 2^-8 of the mean magnitude),
-since their outputs reach |y| ~ 6 where one bf16 ulp is 0.03.
+since their outputs reach |y| ~ 6 where one bf16 ulp is 0.03.  The residual stream of
+the fused add + LayerNorm is compared bit for bit (one rounding of an exact sum).  The
+GELU output adds the error of the epilogue's tanh, taken as at most 2^-10 absolute
+(a hardware tanh approximation's bound), i.e. 2^-10 |a| / 2 for pre-activation a, which
+the magnitude |y| + |a| / 8 covers.
 """
 import math
 
@@ -178,6 +183,181 @@ def test_half_block_graph_capture():
     side.wait_stream(torch.cuda.current_stream())
     with torch.cuda.stream(side):
         run(x0.clone())  # warm-up (plans, algorithms) outside the capture
+    torch.cuda.current_stream().wait_stream(side)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=side):
+        run(xg)
+    xg.copy_(x0)
+    g.replay()
+    torch.cuda.synchronize()
+    assert torch.equal(xg, eager)
+
+
+# MLP hidden width per encoder width: ViT-B/16 3072, ViT-L/14 4096, SigLIP-So400m 4304.
+MLP = {768: 3072, 1024: 4096, 1152: 4304}
+
+
+def mlp_weights(W, F, seed):
+    return {"g2": si.normal_bf16(seed, (W,), 1.0, 0.1), "be2": si.normal_bf16(seed + 1, (W,), 0.0, 0.1),
+            "w1": si.normal_bf16(seed + 2, (F, W), 0.0, 1.0 / math.sqrt(W)),
+            "b1": si.normal_bf16(seed + 3, (F,), 0.0, 0.1),
+            "w2": si.normal_bf16(seed + 4, (W, F), 0.0, 1.0 / math.sqrt(F)),
+            "b2": si.normal_bf16(seed + 5, (W,), 0.0, 0.1)}
+
+
+def gelu_magnitude(x, w, b):
+    """|gelu(a)| + |a| / 8 for the pre-activation a = x @ w.T + b."""
+    a = np.abs(oracle.linear_bf16(x, w, b))
+    return np.abs(oracle.linear_gelu_bf16(x, w, b)) + a / 8.0
+
+
+@pytest.mark.parametrize("name,B,N,H,d", ENCODERS)
+def test_add_layernorm_encoder_widths(name, B, N, H, d):
+    import vit_self_attention_b200 as vab
+    M, W = B * N, H * d
+    x, g, b = ln_inputs(M, W, 900 + W)
+    r = si.normal_bf16(950 + W, (M, W), 0.0, 0.7)
+    s, y = vab.add_layernorm(dev(x), dev(r), dev(g), dev(b), 1e-6)
+    torch.cuda.synchronize()
+    want_s, want_y = oracle.add_layernorm_bf16(x, r, g, b, 1e-6)
+    assert np.array_equal(host(s), want_s), f"residual stream bits, {name}"
+    assert_close_bf16(f64(y), want_y, f"add + LayerNorm {name}")
+
+
+@pytest.mark.parametrize("M,W", [(1, 8), (7, 16), (33, 248), (9, 264), (3, 2048), (1000, 1152)])
+def test_add_layernorm_edge_shapes_and_in_place(M, W):
+    import vit_self_attention_b200 as vab
+    x, g, b = ln_inputs(M, W, 1000 + M + W)
+    r = si.normal_bf16(1001 + M + W, (M, W), 0.0, 3.0)
+    want_s, want_y = oracle.add_layernorm_bf16(x, r, g, b, 1e-5)
+    xt, rt = dev(x), dev(r)
+    s, y = vab.add_layernorm(xt, rt, dev(g), dev(b), 1e-5)
+    torch.cuda.synchronize()
+    assert np.array_equal(host(s), want_s)
+    assert_close_bf16(f64(y), want_y, f"add + LayerNorm M={M} W={W}")
+    vab.add_layernorm(xt, rt, dev(g), dev(b), 1e-5, out_s=xt, out_y=rt)  # both in place
+    torch.cuda.synchronize()
+    assert np.array_equal(host(xt), want_s)
+    assert_close_bf16(f64(rt), want_y, f"add + LayerNorm in place M={M} W={W}")
+
+
+@pytest.mark.parametrize("name,B,N,H,d", ENCODERS)
+def test_linear_gelu_mlp_shapes(name, B, N, H, d):
+    import vit_self_attention_b200 as vab
+    M, K = B * N, H * d
+    F = MLP[K]
+    x, w, b = linear_inputs(M, K, F, 1100 + K)
+    got = vab.linear_gelu(dev(x), dev(w), dev(b))
+    torch.cuda.synchronize()
+    assert_close_bf16(f64(got), oracle.linear_gelu_bf16(x, w, b), f"fc1 + GELU {name}",
+                      mag=gelu_magnitude(x, w, b))
+
+
+@pytest.mark.parametrize("M,K,N,bias", [(1, 8, 8, True), (5, 16, 24, False), (77, 64, 200, True),
+                                        (300, 1152, 4304, False)])
+def test_linear_gelu_variants(M, K, N, bias):
+    import vit_self_attention_b200 as vab
+    x, w, b = linear_inputs(M, K, N, 1200 + M + K + N)
+    b = b if bias else None
+    got = vab.linear_gelu(dev(x), dev(w), dev(b) if bias else None)
+    torch.cuda.synchronize()
+    assert_close_bf16(f64(got), oracle.linear_gelu_bf16(x, w, b),
+                      f"linear + GELU M={M} K={K} N={N} bias={bias}", mag=gelu_magnitude(x, w, b))
+
+
+def _layer_stagewise(cfg, fused_norm):
+    """One pre-norm encoder layer on the GPU, each stage against the oracle on the GPU's
+    own bf16 input to that stage.  fused_norm: the output projection leaves the residual
+    to the fused add + LayerNorm; otherwise it adds it in its epilogue and LN2 is plain."""
+    import vit_self_attention_b200 as vab
+    c = si.CONFIGS[cfg]
+    W = c.H * c.d
+    F = MLP[W]
+    x = si.normal_bf16(1300 + cfg, (c.B, c.N, W))
+    p = {**block_weights(W, 1310 + cfg), **mlp_weights(W, F, 1320 + cfg)}
+    t = {k: dev(v) for k, v in p.items()}
+    xt = dev(x)
+    xn = vab.layernorm(xt, t["g"], t["be"], 1e-6)
+    qkv = vab.linear(xn, t["wqkv"], t["bqkv"])
+    o = vab.attention(qkv.view(c.B, c.N, 3, c.H, c.d), c.scale)
+    if fused_norm:
+        proj = vab.linear(o.view(c.B, c.N, W), t["wo"], t["bo"])
+        h, hn = vab.add_layernorm(xt, proj, t["g2"], t["be2"], 1e-6)
+    else:
+        h = vab.linear(o.view(c.B, c.N, W), t["wo"], t["bo"], xt)
+        hn = vab.layernorm(h, t["g2"], t["be2"], 1e-6)
+    a = vab.linear_gelu(hn, t["w1"], t["b1"])
+    out = vab.linear(a, t["w2"], t["b2"], h)
+    torch.cuda.synchronize()
+    assert_close_bf16(f64(xn), oracle.layernorm_bf16(x, p["g"], p["be"], 1e-6), "LN1")
+    assert_close_bf16(f64(qkv), oracle.linear_bf16(host(xn), p["wqkv"], p["bqkv"]), "qkv")
+    assert_parity(f64(o), oracle.attention_packed_bf16(host(qkv).reshape(c.B, c.N, 3, c.H, c.d),
+                                                       c.scale), "attention")
+    ob = host(o).reshape(c.B, c.N, W)
+    if fused_norm:
+        assert_close_bf16(f64(proj), oracle.linear_bf16(ob, p["wo"], p["bo"]), "output projection",
+                          mag=residual_magnitude(ob, p["wo"], p["bo"], None))
+        want_h, want_hn = oracle.add_layernorm_bf16(x, host(proj), p["g2"], p["be2"], 1e-6)
+        assert np.array_equal(host(h), want_h), "residual stream after attention"
+        assert_close_bf16(f64(hn), want_hn, "add + LN2")
+    else:
+        assert_close_bf16(f64(h), oracle.linear_bf16(ob, p["wo"], p["bo"], x),
+                          "output projection + residual",
+                          mag=residual_magnitude(ob, p["wo"], p["bo"], x))
+        assert_close_bf16(f64(hn), oracle.layernorm_bf16(host(h), p["g2"], p["be2"], 1e-6), "LN2")
+    hb = host(hn)
+    assert_close_bf16(f64(a), oracle.linear_gelu_bf16(hb, p["w1"], p["b1"]), "fc1 + GELU",
+                      mag=gelu_magnitude(hb, p["w1"], p["b1"]))
+    ab, hh = host(a), host(h)
+    assert_close_bf16(f64(out), oracle.linear_bf16(ab, p["w2"], p["b2"], hh), "fc2 + residual",
+                      mag=residual_magnitude(ab, p["w2"], p["b2"], hh))
+
+
+@pytest.mark.parametrize("cfg", [0, 1, 3])
+def test_encoder_layer_stagewise(cfg):
+    _layer_stagewise(cfg, fused_norm=False)
+
+
+@pytest.mark.parametrize("cfg", [1, 3])
+def test_encoder_layer_stagewise_fused_residual_norm(cfg):
+    _layer_stagewise(cfg, fused_norm=True)
+
+
+def test_encoder_layers_graph_capture():
+    """Two whole encoder layers captured in one CUDA graph and replayed give the eager
+    bytes."""
+    import vit_self_attention_b200 as vab
+    c = si.CONFIGS[3]
+    W = c.H * c.d
+    F = MLP[W]
+    x0 = dev(si.normal_bf16(1400, (c.B, c.N, W)))
+    layers = [{k: dev(v) for k, v in {**block_weights(W, 1410 + 10 * i),
+                                       **mlp_weights(W, F, 1450 + 10 * i)}.items()}
+              for i in range(2)]
+    ws = torch.empty(vab.vla_linear_workspace_bytes(), dtype=torch.uint8, device="cuda")
+    e = lambda *shape: torch.empty(shape, dtype=torch.bfloat16, device="cuda")
+    bufs = {"xn": e(c.B, c.N, W), "qkv": e(c.B, c.N, 3 * W), "o": e(c.B, c.N, c.H, c.d),
+            "a": e(c.B, c.N, F)}
+
+    def run(x):
+        for p in layers:
+            vab.layernorm(x, p["g"], p["be"], 1e-6, out=bufs["xn"])
+            vab.linear(bufs["xn"], p["wqkv"], p["bqkv"], out=bufs["qkv"], workspace=ws)
+            vab.attention(bufs["qkv"].view(c.B, c.N, 3, c.H, c.d), c.scale, out=bufs["o"])
+            vab.linear(bufs["o"].view(c.B, c.N, W), p["wo"], p["bo"], x, out=x, workspace=ws)
+            vab.layernorm(x, p["g2"], p["be2"], 1e-6, out=bufs["xn"])
+            vab.linear_gelu(bufs["xn"], p["w1"], p["b1"], out=bufs["a"], workspace=ws)
+            vab.linear(bufs["a"], p["w2"], p["b2"], x, out=x, workspace=ws)
+
+    eager = x0.clone()
+    run(eager)
+    torch.cuda.synchronize()
+    xg = x0.clone()
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        run(x0.clone())
     torch.cuda.current_stream().wait_stream(side)
     torch.cuda.synchronize()
     g = torch.cuda.CUDAGraph()

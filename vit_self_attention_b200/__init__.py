@@ -52,6 +52,10 @@ _lib.vla_linear_fwd.argtypes = [_VP, _VP, _VP, _VP, _VP, _I, _I, _I, _VP, ctypes
 _lib.vla_linear_fwd.restype = _I
 _lib.vla_linear_workspace_bytes.argtypes = []
 _lib.vla_linear_workspace_bytes.restype = ctypes.c_size_t
+_lib.vla_add_layernorm_fwd.argtypes = [_VP, _VP, _VP, _VP, _VP, _VP, _I, _I, ctypes.c_float, _VP]
+_lib.vla_add_layernorm_fwd.restype = _I
+_lib.vla_linear_gelu_fwd.argtypes = [_VP, _VP, _VP, _VP, _I, _I, _I, _VP, ctypes.c_size_t, _VP]
+_lib.vla_linear_gelu_fwd.restype = _I
 _lib.vla_linear_fwd_static.argtypes = [_VP, _VP, _VP, _VP, _VP, _I, _I, _I, _VP]
 _lib.vla_linear_fwd_static.restype = _I
 _lib.vla_linear_static_workspace_bytes.argtypes = []
@@ -74,7 +78,8 @@ EXPORTED_SYMBOLS = (
     "vla_attn_reset_device_status", "vla_attn_max_tokens", "vla_attn_launch_count",
     "vla_attn_set_wait_limit_ns",
     "vla_attn_set_test_stall", "vla_layernorm_fwd", "vla_linear_fwd", "vla_linear_workspace_bytes",
-    "vla_linear_fwd_static", "vla_linear_static_workspace_bytes",
+    "vla_linear_fwd_static", "vla_linear_static_workspace_bytes", "vla_add_layernorm_fwd",
+    "vla_linear_gelu_fwd",
 )
 
 
@@ -165,6 +170,26 @@ def vla_layernorm_fwd(x, gamma, beta, y, M: int, W: int, eps: float, stream=None
     return st
 
 
+def vla_add_layernorm_fwd(x, r, gamma, beta, s, y, M: int, W: int, eps: float, stream=None,
+                          check: bool = True) -> int:
+    """Enqueue ``s = bf16(x + r)``, ``y = LayerNorm(s)`` (see include/vla_attn.h)."""
+    st = _lib.vla_add_layernorm_fwd(_addr(x), _addr(r), _addr(gamma), _addr(beta), _addr(s),
+                                    _addr(y), int(M), int(W), float(eps), _stream(stream))
+    if check and st != OK:
+        raise VlaAttnError(st)
+    return st
+
+
+def vla_linear_gelu_fwd(x, w, bias, y, M: int, K: int, N: int, workspace=None,
+                        workspace_bytes: int = 0, stream=None, check: bool = True) -> int:
+    """Enqueue ``y = gelu(x @ w.T + bias)`` (tanh GELU; see include/vla_attn.h)."""
+    st = _lib.vla_linear_gelu_fwd(_addr(x), _addr(w), _addr(bias), _addr(y), int(M), int(K),
+                                  int(N), _addr(workspace), int(workspace_bytes), _stream(stream))
+    if check and st != OK:
+        raise VlaAttnError(st)
+    return st
+
+
 def vla_linear_workspace_bytes() -> int:
     return int(_lib.vla_linear_workspace_bytes())
 
@@ -207,6 +232,35 @@ def layernorm(x, gamma, beta, eps: float = 1e-6, out=None, stream=None):
     return out
 
 
+def add_layernorm(x, r, gamma, beta, eps: float = 1e-6, out_s=None, out_y=None, stream=None):
+    """``(s, y)``: the residual stream ``s = bf16(x + r)`` and ``y = LayerNorm(s)`` for
+    contiguous bf16 CUDA tensors of one shape (``out_s`` may be ``x`` or ``r``)."""
+    import torch
+    for t in (x, r):
+        if t.dtype != torch.bfloat16 or not t.is_cuda or not t.is_contiguous():
+            raise ValueError("x and r must be contiguous bf16 CUDA tensors")
+    if x.shape != r.shape:
+        raise ValueError("x and r must have one shape")
+    W = int(x.shape[-1])
+    s = torch.empty_like(x) if out_s is None else out_s
+    y = torch.empty_like(x) if out_y is None else out_y
+    vla_add_layernorm_fwd(x, r, gamma, beta, s, y, x.numel() // W, W, eps, stream)
+    return s, y
+
+
+def linear_gelu(x, w, bias=None, out=None, workspace=None, stream=None):
+    """``gelu(x @ w.T + bias)`` (tanh GELU) for contiguous bf16 CUDA tensors."""
+    import torch
+    N, K = (int(v) for v in w.shape)
+    M = x.numel() // K
+    if out is None:
+        out = torch.empty(tuple(x.shape[:-1]) + (N,), dtype=torch.bfloat16, device=x.device)
+    if workspace is None:
+        workspace = torch.empty(vla_linear_workspace_bytes(), dtype=torch.uint8, device=x.device)
+    vla_linear_gelu_fwd(x, w, bias, out, M, K, N, workspace, workspace.numel(), stream)
+    return out
+
+
 def linear(x, w, bias=None, res=None, out=None, workspace=None, stream=None):
     """``x @ w.T + bias (+ res)`` for contiguous bf16 CUDA tensors (``w`` is ``[N, K]``)."""
     import torch
@@ -244,6 +298,6 @@ __all__ = [
     "vla_attn_strerror", "vla_attn_last_device_status", "vla_attn_reset_device_status",
     "vla_attn_max_tokens", "vla_attn_launch_count", "vla_attn_set_wait_limit_ns",
     "vla_attn_set_test_stall", "vla_layernorm_fwd", "vla_linear_fwd", "vla_linear_workspace_bytes",
-    "vla_linear_fwd_static", "vla_linear_static_workspace_bytes", "layernorm", "linear",
-    "attention",
+    "vla_linear_fwd_static", "vla_linear_static_workspace_bytes", "vla_add_layernorm_fwd",
+    "vla_linear_gelu_fwd", "layernorm", "add_layernorm", "linear", "linear_gelu", "attention",
 ]

@@ -1,6 +1,7 @@
-// The layers on either side of the attention core in a ViT block: the
-// LayerNorm before the qkv linear, and the linear layers themselves (qkv
-// projection, output projection with the residual add).
+// The layers around the attention core in a ViT encoder layer: the
+// LayerNorms (plain, or fused with the residual add), the linear layers (qkv
+// projection, output projection with the residual add, the MLP's fc1 with
+// its GELU and fc2 with the residual add).
 //
 //   LayerNorm over the last dimension (width W) of every row, biased
 //   variance, fp32 statistics:
@@ -9,7 +10,9 @@
 //   fusion, residual add + LayerNorm in one kernel.)  A hand-written kernel:
 //   one warp per row, 16-byte loads, the row kept in registers between the
 //   mean, the variance and the output pass, so x is read once and y written
-//   once (HBM-bound).
+//   once (HBM-bound).  The fused variant first forms the residual stream
+//   s = bf16(x + r), stores it, and normalises the stored values, so that it
+//   gives exactly what a separate add and LayerNorm give.
 //
 //   Linear layer with bias and optional residual, nn.Linear weight layout
 //   [N, K] (the pages' weight(K,N) transposed):
@@ -21,6 +24,8 @@
 //   residual as C with beta = 1); the row-major product is computed as the
 //   column-major y^T = w . x^T.  For the qkv linear, N = 3 H d and y is
 //   exactly the packed [B, tokens, 3, H, d] input of the attention kernel.
+//   The MLP's first layer applies GELU (the tanh form) in the same epilogue
+//   (same page, Triton fused kernels: matrix multiply + bias + activation).
 //
 // This header is included by vla_attn.cu after its host helpers (device
 // checks, pointer-range checks) and shares them.
@@ -52,24 +57,59 @@ __device__ __forceinline__ void unpack8(const uint4& u, float (&f)[8]) {
 
 // One warp per row; lane l holds elements [256 c + 8 l, 256 c + 8 l + 8) of
 // chunk c < NCH (elements at or past W are skipped).  8 rows per block.
-template <int NCH>
-__global__ void __launch_bounds__(256) layernorm_kernel(const __nv_bfloat16* __restrict__ x,
+// ADD: the row is first the residual sum s = bf16(x + r), stored to `s` and
+// then normalised (the stream as stored, so the fusion changes no result).
+// A row is entirely in registers before any of its outputs is written, and
+// rows belong to one warp each, so an output may be the very buffer x or r.
+template <int NCH, bool ADD>
+__global__ void __launch_bounds__(256) layernorm_kernel(const __nv_bfloat16* x,
+                                                        const __nv_bfloat16* r,
                                                         const __nv_bfloat16* __restrict__ gamma,
                                                         const __nv_bfloat16* __restrict__ beta,
-                                                        __nv_bfloat16* y, long long M, int W,
-                                                        float eps) {
+                                                        __nv_bfloat16* s, __nv_bfloat16* y,
+                                                        long long M, int W, float eps) {
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const long long row = static_cast<long long>(blockIdx.x) * 8 + warp;
   if (row >= M) return;
   const __nv_bfloat16* xr = x + row * W;
   float v[NCH][8];
+  uint4 sum_bits[ADD ? NCH : 1];
+  if constexpr (ADD) {
+    const __nv_bfloat16* rr = r + row * W;
+    uint4 xb[NCH], rb[NCH];
+#pragma unroll
+    for (int c = 0; c < NCH; ++c) {  // all loads of the row first
+      const int e = c * 256 + lane * 8;
+      if (e < W) {
+        xb[c] = *reinterpret_cast<const uint4*>(xr + e);
+        rb[c] = *reinterpret_cast<const uint4*>(rr + e);
+      }
+    }
+#pragma unroll
+    for (int c = 0; c < NCH; ++c) {
+      if (c * 256 + lane * 8 < W) {
+        float a[8], b[8];
+        unpack8(xb[c], a);
+        unpack8(rb[c], b);
+        uint32_t o[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) o[i] = pack_bf16x2(a[2 * i] + b[2 * i], a[2 * i + 1] + b[2 * i + 1]);
+        sum_bits[c] = make_uint4(o[0], o[1], o[2], o[3]);
+        unpack8(sum_bits[c], v[c]);
+      }
+    }
+  } else {
+#pragma unroll
+    for (int c = 0; c < NCH; ++c) {
+      const int e = c * 256 + lane * 8;
+      if (e < W) unpack8(*reinterpret_cast<const uint4*>(xr + e), v[c]);
+    }
+  }
   float sum = 0.0f;
 #pragma unroll
   for (int c = 0; c < NCH; ++c) {
-    const int e = c * 256 + lane * 8;
-    if (e < W) {
-      unpack8(*reinterpret_cast<const uint4*>(xr + e), v[c]);
+    if (c * 256 + lane * 8 < W) {
 #pragma unroll
       for (int i = 0; i < 8; ++i) sum += v[c][i];
     }
@@ -92,6 +132,7 @@ __global__ void __launch_bounds__(256) layernorm_kernel(const __nv_bfloat16* __r
   for (int c = 0; c < NCH; ++c) {
     const int e = c * 256 + lane * 8;
     if (e < W) {
+      if constexpr (ADD) *reinterpret_cast<uint4*>(s + row * W + e) = sum_bits[c];
       float g[8], b[8];
       unpack8(*reinterpret_cast<const uint4*>(gamma + e), g);
       unpack8(*reinterpret_cast<const uint4*>(beta + e), b);
@@ -117,16 +158,32 @@ bool overlaps(uintptr_t a_lo, uintptr_t a_hi, uintptr_t b_lo, uintptr_t b_hi) {
   return a_lo < b_hi && b_lo < a_hi;
 }
 
-template <int NCH>
-int launch_layernorm(const void* x, const void* gamma, const void* beta, void* y, long long M,
-                     int W, float eps, cudaStream_t stream) {
+template <int NCH, bool ADD>
+int launch_layernorm(const void* x, const void* r, const void* gamma, const void* beta, void* s,
+                     void* y, long long M, int W, float eps, cudaStream_t stream) {
   const long long blocks = (M + 7) / 8;
-  vla::layernorm_kernel<NCH><<<static_cast<unsigned>(blocks), 256, 0, stream>>>(
-      static_cast<const __nv_bfloat16*>(x), static_cast<const __nv_bfloat16*>(gamma),
-      static_cast<const __nv_bfloat16*>(beta), static_cast<__nv_bfloat16*>(y), M, W, eps);
+  vla::layernorm_kernel<NCH, ADD><<<static_cast<unsigned>(blocks), 256, 0, stream>>>(
+      static_cast<const __nv_bfloat16*>(x), static_cast<const __nv_bfloat16*>(r),
+      static_cast<const __nv_bfloat16*>(gamma), static_cast<const __nv_bfloat16*>(beta),
+      static_cast<__nv_bfloat16*>(s), static_cast<__nv_bfloat16*>(y), M, W, eps);
   if (cudaGetLastError() != cudaSuccess) return VLA_ATTN_ERR_CUDA;
   g_launches.fetch_add(1);
   return VLA_ATTN_OK;
+}
+
+template <bool ADD>
+int dispatch_layernorm(const void* x, const void* r, const void* gamma, const void* beta, void* s,
+                       void* y, long long M, int W, float eps, cudaStream_t st) {
+  switch ((W + 255) / 256) {
+    case 1: return launch_layernorm<1, ADD>(x, r, gamma, beta, s, y, M, W, eps, st);
+    case 2: return launch_layernorm<2, ADD>(x, r, gamma, beta, s, y, M, W, eps, st);
+    case 3: return launch_layernorm<3, ADD>(x, r, gamma, beta, s, y, M, W, eps, st);
+    case 4: return launch_layernorm<4, ADD>(x, r, gamma, beta, s, y, M, W, eps, st);
+    case 5: return launch_layernorm<5, ADD>(x, r, gamma, beta, s, y, M, W, eps, st);
+    case 6: return launch_layernorm<6, ADD>(x, r, gamma, beta, s, y, M, W, eps, st);
+    case 7: return launch_layernorm<7, ADD>(x, r, gamma, beta, s, y, M, W, eps, st);
+    default: return launch_layernorm<8, ADD>(x, r, gamma, beta, s, y, M, W, eps, st);
+  }
 }
 
 // cuBLASLt state: one handle per process, one plan (descriptors + heuristic
@@ -139,12 +196,14 @@ struct LtPlan {
 
 std::mutex g_lt_mutex;
 cublasLtHandle_t g_lt = nullptr;
-std::map<std::tuple<int, int, int, int, int, int, size_t>, LtPlan> g_lt_plans;
+std::map<std::tuple<int, int, int, int, int, int, int, size_t>, LtPlan> g_lt_plans;
 
-// Builds (once) the plan of y^T[N, M] = w[N, K] . x^T[K, M] (+ bias) (+ res^T).
-int lt_plan(int dev, int M, int K, int N, bool bias, bool res, size_t ws, LtPlan** out) {
+// Builds (once) the plan of y^T[N, M] = act(w[N, K] . x^T[K, M] (+ bias)) (+ res^T),
+// act = GELU (cuBLASLt's epilogue, the tanh form) or the identity.
+int lt_plan(int dev, int M, int K, int N, bool bias, bool res, bool gelu, size_t ws,
+            LtPlan** out) {
   if (g_lt == nullptr && cublasLtCreate(&g_lt) != CUBLAS_STATUS_SUCCESS) return VLA_ATTN_ERR_CUDA;
-  const auto key = std::make_tuple(dev, M, K, N, bias ? 1 : 0, res ? 1 : 0, ws);
+  const auto key = std::make_tuple(dev, M, K, N, bias ? 1 : 0, res ? 1 : 0, gelu ? 1 : 0, ws);
   auto it = g_lt_plans.find(key);
   if (it != g_lt_plans.end()) {
     *out = &it->second;
@@ -154,7 +213,9 @@ int lt_plan(int dev, int M, int K, int N, bool bias, bool res, size_t ws, LtPlan
   bool ok = cublasLtMatmulDescCreate(&pl.op, CUBLAS_COMPUTE_32F, CUDA_R_32F) ==
             CUBLAS_STATUS_SUCCESS;
   const cublasOperation_t ta = CUBLAS_OP_T, tb = CUBLAS_OP_N;
-  const cublasLtEpilogue_t epi = bias ? CUBLASLT_EPILOGUE_BIAS : CUBLASLT_EPILOGUE_DEFAULT;
+  const cublasLtEpilogue_t epi =
+      gelu ? (bias ? CUBLASLT_EPILOGUE_GELU_BIAS : CUBLASLT_EPILOGUE_GELU)
+           : (bias ? CUBLASLT_EPILOGUE_BIAS : CUBLASLT_EPILOGUE_DEFAULT);
   const cudaDataType_t bias_type = CUDA_R_16BF;
   ok = ok && cublasLtMatmulDescSetAttribute(pl.op, CUBLASLT_MATMUL_DESC_TRANSA, &ta,
                                             sizeof(ta)) == CUBLAS_STATUS_SUCCESS;
@@ -220,64 +281,10 @@ int static_workspace(int dev, void** out) {
   return VLA_ATTN_OK;
 }
 
-}  // namespace
-
-extern "C" {
-
-int vla_layernorm_fwd(const void* x, const void* gamma, const void* beta, void* y, int M, int W,
-                      float eps, void* stream) {
-  if (x == nullptr || gamma == nullptr || beta == nullptr || y == nullptr) return VLA_ATTN_ERR_NULL;
-  if (M < 1 || W < 1) return VLA_ATTN_ERR_SHAPE;
-  if (W % 8 != 0 || W > 256 * vla::kLnMaxChunks) return VLA_ATTN_ERR_UNSUPPORTED;
-  if (!std::isfinite(eps) || eps < 0.0f) return VLA_ATTN_ERR_SCALE;
-  if (!aligned16(x) || !aligned16(gamma) || !aligned16(beta) || !aligned16(y))
-    return VLA_ATTN_ERR_ALIGN;
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return VLA_ATTN_ERR_CUDA;
-  DeviceInfo di;
-  int rc = device_info(dev, &di);
-  if (rc != VLA_ATTN_OK) return rc;
-  const DriverFns& fns = driver_fns();
-  if (fns.ptr_attr == nullptr) return VLA_ATTN_ERR_CUDA;
-  const size_t bytes = static_cast<size_t>(M) * W * 2u;
-  uintptr_t xl, xh, yl, yh, gl, gh, bl, bh;
-  if ((rc = check_device_range(fns, x, bytes, dev, &xl, &xh)) != VLA_ATTN_OK) return rc;
-  if ((rc = check_device_range(fns, y, bytes, dev, &yl, &yh)) != VLA_ATTN_OK) return rc;
-  if ((rc = check_device_range(fns, gamma, W * 2u, dev, &gl, &gh)) != VLA_ATTN_OK) return rc;
-  if ((rc = check_device_range(fns, beta, W * 2u, dev, &bl, &bh)) != VLA_ATTN_OK) return rc;
-  // In place (y == x) is allowed: a row is in registers before it is written.
-  if ((y != x && overlaps(xl, xh, yl, yh)) || overlaps(gl, gh, yl, yh) || overlaps(bl, bh, yl, yh))
-    return VLA_ATTN_ERR_MEMORY;
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
-  switch ((W + 255) / 256) {
-    case 1: return launch_layernorm<1>(x, gamma, beta, y, M, W, eps, s);
-    case 2: return launch_layernorm<2>(x, gamma, beta, y, M, W, eps, s);
-    case 3: return launch_layernorm<3>(x, gamma, beta, y, M, W, eps, s);
-    case 4: return launch_layernorm<4>(x, gamma, beta, y, M, W, eps, s);
-    case 5: return launch_layernorm<5>(x, gamma, beta, y, M, W, eps, s);
-    case 6: return launch_layernorm<6>(x, gamma, beta, y, M, W, eps, s);
-    case 7: return launch_layernorm<7>(x, gamma, beta, y, M, W, eps, s);
-    default: return launch_layernorm<8>(x, gamma, beta, y, M, W, eps, s);
-  }
-}
-
-size_t vla_linear_workspace_bytes(void) { return kLinearWorkspaceBytes; }
-
-size_t vla_linear_static_workspace_bytes(void) { return kStaticWorkspaceBytes; }
-
-int vla_linear_fwd_static(const void* x, const void* w, const void* bias, const void* res, void* y,
-                          int M, int K, int N, void* stream) {
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return VLA_ATTN_ERR_CUDA;
-  if (dev < 0 || dev >= kMaxDevices) return VLA_ATTN_ERR_DEVICE;
-  void* ws = nullptr;
-  const int rc = static_workspace(dev, &ws);
-  if (rc != VLA_ATTN_OK) return rc;
-  return vla_linear_fwd(x, w, bias, res, y, M, K, N, ws, kStaticWorkspaceBytes, stream);
-}
-
-int vla_linear_fwd(const void* x, const void* w, const void* bias, const void* res, void* y,
-                   int M, int K, int N, void* workspace, size_t workspace_bytes, void* stream) {
+// y = act(x . w^T + bias) (+ res) through one cuBLASLt matmul; argument checks
+// of vla_linear_fwd.
+int linear_impl(const void* x, const void* w, const void* bias, const void* res, void* y, int M,
+                int K, int N, void* workspace, size_t workspace_bytes, void* stream, bool gelu) {
   if (x == nullptr || w == nullptr || y == nullptr) return VLA_ATTN_ERR_NULL;
   if (workspace == nullptr && workspace_bytes != 0) return VLA_ATTN_ERR_NULL;
   if (M < 1 || K < 1 || N < 1) return VLA_ATTN_ERR_SHAPE;
@@ -315,7 +322,7 @@ int vla_linear_fwd(const void* x, const void* w, const void* bias, const void* r
 
   std::lock_guard<std::mutex> lock(g_lt_mutex);
   LtPlan* pl = nullptr;
-  rc = lt_plan(dev, M, K, N, bias != nullptr, res != nullptr, workspace_bytes, &pl);
+  rc = lt_plan(dev, M, K, N, bias != nullptr, res != nullptr, gelu, workspace_bytes, &pl);
   if (rc != VLA_ATTN_OK) return rc;
   if (bias != nullptr &&
       cublasLtMatmulDescSetAttribute(pl->op, CUBLASLT_MATMUL_DESC_BIAS_POINTER, &bias,
@@ -329,6 +336,104 @@ int vla_linear_fwd(const void* x, const void* w, const void* bias, const void* r
                      static_cast<cudaStream_t>(stream)) != CUBLAS_STATUS_SUCCESS)
     return VLA_ATTN_ERR_CUDA;
   return VLA_ATTN_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int vla_layernorm_fwd(const void* x, const void* gamma, const void* beta, void* y, int M, int W,
+                      float eps, void* stream) {
+  if (x == nullptr || gamma == nullptr || beta == nullptr || y == nullptr) return VLA_ATTN_ERR_NULL;
+  if (M < 1 || W < 1) return VLA_ATTN_ERR_SHAPE;
+  if (W % 8 != 0 || W > 256 * vla::kLnMaxChunks) return VLA_ATTN_ERR_UNSUPPORTED;
+  if (!std::isfinite(eps) || eps < 0.0f) return VLA_ATTN_ERR_SCALE;
+  if (!aligned16(x) || !aligned16(gamma) || !aligned16(beta) || !aligned16(y))
+    return VLA_ATTN_ERR_ALIGN;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return VLA_ATTN_ERR_CUDA;
+  DeviceInfo di;
+  int rc = device_info(dev, &di);
+  if (rc != VLA_ATTN_OK) return rc;
+  const DriverFns& fns = driver_fns();
+  if (fns.ptr_attr == nullptr) return VLA_ATTN_ERR_CUDA;
+  const size_t bytes = static_cast<size_t>(M) * W * 2u;
+  uintptr_t xl, xh, yl, yh, gl, gh, bl, bh;
+  if ((rc = check_device_range(fns, x, bytes, dev, &xl, &xh)) != VLA_ATTN_OK) return rc;
+  if ((rc = check_device_range(fns, y, bytes, dev, &yl, &yh)) != VLA_ATTN_OK) return rc;
+  if ((rc = check_device_range(fns, gamma, W * 2u, dev, &gl, &gh)) != VLA_ATTN_OK) return rc;
+  if ((rc = check_device_range(fns, beta, W * 2u, dev, &bl, &bh)) != VLA_ATTN_OK) return rc;
+  // In place (y == x) is allowed: a row is in registers before it is written.
+  if ((y != x && overlaps(xl, xh, yl, yh)) || overlaps(gl, gh, yl, yh) || overlaps(bl, bh, yl, yh))
+    return VLA_ATTN_ERR_MEMORY;
+  return dispatch_layernorm<false>(x, nullptr, gamma, beta, nullptr, y, M, W, eps,
+                                   static_cast<cudaStream_t>(stream));
+}
+
+int vla_add_layernorm_fwd(const void* x, const void* r, const void* gamma, const void* beta,
+                          void* s, void* y, int M, int W, float eps, void* stream) {
+  if (x == nullptr || r == nullptr || gamma == nullptr || beta == nullptr || s == nullptr ||
+      y == nullptr)
+    return VLA_ATTN_ERR_NULL;
+  if (M < 1 || W < 1) return VLA_ATTN_ERR_SHAPE;
+  if (W % 8 != 0 || W > 256 * vla::kLnMaxChunks) return VLA_ATTN_ERR_UNSUPPORTED;
+  if (!std::isfinite(eps) || eps < 0.0f) return VLA_ATTN_ERR_SCALE;
+  if (!aligned16(x) || !aligned16(r) || !aligned16(gamma) || !aligned16(beta) || !aligned16(s) ||
+      !aligned16(y))
+    return VLA_ATTN_ERR_ALIGN;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return VLA_ATTN_ERR_CUDA;
+  DeviceInfo di;
+  int rc = device_info(dev, &di);
+  if (rc != VLA_ATTN_OK) return rc;
+  const DriverFns& fns = driver_fns();
+  if (fns.ptr_attr == nullptr) return VLA_ATTN_ERR_CUDA;
+  const size_t bytes = static_cast<size_t>(M) * W * 2u;
+  uintptr_t xl, xh, rl, rh, sl, sh, yl, yh, gl, gh, bl, bh;
+  if ((rc = check_device_range(fns, x, bytes, dev, &xl, &xh)) != VLA_ATTN_OK) return rc;
+  if ((rc = check_device_range(fns, r, bytes, dev, &rl, &rh)) != VLA_ATTN_OK) return rc;
+  if ((rc = check_device_range(fns, s, bytes, dev, &sl, &sh)) != VLA_ATTN_OK) return rc;
+  if ((rc = check_device_range(fns, y, bytes, dev, &yl, &yh)) != VLA_ATTN_OK) return rc;
+  if ((rc = check_device_range(fns, gamma, W * 2u, dev, &gl, &gh)) != VLA_ATTN_OK) return rc;
+  if ((rc = check_device_range(fns, beta, W * 2u, dev, &bl, &bh)) != VLA_ATTN_OK) return rc;
+  // Each output is either exactly x or r, or disjoint from them; the two
+  // outputs are disjoint; gamma and beta are disjoint from both outputs.
+  const void* outs[2] = {s, y};
+  const uintptr_t olo[2] = {sl, yl}, ohi[2] = {sh, yh};
+  for (int i = 0; i < 2; ++i) {
+    if ((outs[i] != x && overlaps(xl, xh, olo[i], ohi[i])) ||
+        (outs[i] != r && overlaps(rl, rh, olo[i], ohi[i])) || overlaps(gl, gh, olo[i], ohi[i]) ||
+        overlaps(bl, bh, olo[i], ohi[i]))
+      return VLA_ATTN_ERR_MEMORY;
+  }
+  if (overlaps(sl, sh, yl, yh)) return VLA_ATTN_ERR_MEMORY;
+  return dispatch_layernorm<true>(x, r, gamma, beta, s, y, M, W, eps,
+                                  static_cast<cudaStream_t>(stream));
+}
+
+size_t vla_linear_workspace_bytes(void) { return kLinearWorkspaceBytes; }
+
+size_t vla_linear_static_workspace_bytes(void) { return kStaticWorkspaceBytes; }
+
+int vla_linear_fwd_static(const void* x, const void* w, const void* bias, const void* res, void* y,
+                          int M, int K, int N, void* stream) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return VLA_ATTN_ERR_CUDA;
+  if (dev < 0 || dev >= kMaxDevices) return VLA_ATTN_ERR_DEVICE;
+  void* ws = nullptr;
+  const int rc = static_workspace(dev, &ws);
+  if (rc != VLA_ATTN_OK) return rc;
+  return vla_linear_fwd(x, w, bias, res, y, M, K, N, ws, kStaticWorkspaceBytes, stream);
+}
+
+int vla_linear_fwd(const void* x, const void* w, const void* bias, const void* res, void* y,
+                   int M, int K, int N, void* workspace, size_t workspace_bytes, void* stream) {
+  return linear_impl(x, w, bias, res, y, M, K, N, workspace, workspace_bytes, stream, false);
+}
+
+int vla_linear_gelu_fwd(const void* x, const void* w, const void* bias, void* y, int M, int K,
+                        int N, void* workspace, size_t workspace_bytes, void* stream) {
+  return linear_impl(x, w, bias, nullptr, y, M, K, N, workspace, workspace_bytes, stream, true);
 }
 
 }  // extern "C"
