@@ -80,11 +80,14 @@ def test_longest_sequence_sampled_rows():
 @pytest.mark.parametrize("B,H,N,d", [(8, 4, 577, 64), (4, 5, 1025, 64), (6, 5, 600, 72),
                                      (160, 1, 197, 64), (10, 16, 257, 64), (12, 13, 577, 64),
                                      (75, 2, 577, 72), (1, 1, 577, 64), (148, 1, 129, 72),
-                                     (300, 1, 50, 64)])
+                                     (300, 1, 50, 64), (10, 16, 1025, 64), (149, 1, 577, 64),
+                                     (297, 1, 300, 64), (157, 1, 600, 72)])
 def test_schedules(B, H, N, d):
     """Whole-head work units (B*H >= #SMs), per-round units (fewer heads, more tiles than
     SMs; includes K/V streaming at N > 768 / d=72 N > 560), single-tile units (all tiles
-    fit on the SMs), and persistent multi-unit CTAs."""
+    fit on the SMs), persistent multi-unit CTAs, and stream mode (whole heads with an odd
+    tile count: tiles paired across head boundaries, a lone last tile on CTAs with an odd
+    tile total, K/V streamed, with and without the long-sequence ring wrap)."""
     bits = si.packed_qkv(B, N, H, d, seed=90000 + B * 7 + H * 3 + N + d)
     scale = 1.0 / math.sqrt(d)
     want = oracle.attention_packed_bf16(bits, scale)

@@ -25,12 +25,22 @@
 //               16-byte stores.
 //   warp 3      idle.
 //
+// Schedule.  A round holds up to two 128-row Q tiles, one per Q slot and
+// softmax warpgroup.  With fewer heads than SMs a CTA takes single tiles or
+// single rounds; with more, whole heads, loading a head's K/V once for all its
+// rounds when they fit the ring.  When a head has an odd number of Q tiles
+// (577 tokens make 5), whole-head rounds would end every head with a half
+// round, so instead a CTA walks the tiles of its heads two at a time across
+// head boundaries: the round that pairs the last tile of one head with the
+// first of the next streams both heads' K/V blocks through the ring (one load
+// per slot and block), the others one load per block shared by both slots.
+//
 // Pipelining.  A softmax thread signals "S consumed" as soon as it has the S
 // row of block j in registers, so the tensor core computes S of block j+1
 // while block j is being exponentiated; P V of block j follows as soon as P
 // is stored.  A full round holds two Q tiles of one head (slots 0 and 1, one
 // per softmax warpgroup) whose exponentials share the special-function pipe.
-// A half round (the odd last tile of a head) has slot 0 only.
+// A half round (a lone last tile) has slot 0 only.
 //
 // Tensor memory (512 columns): slot s owns columns [256 s, 256 s + 256):
 // S at +0 (BK fp32 columns), O at +BK (DP = 64 or 80 fp32 columns), P at
@@ -141,6 +151,8 @@ struct AttnParams {
   float c;                 // scale * log2(e)
   unsigned long long wait_limit_ns;
   int test_stall;          // testing hook: softmax warps wait on a barrier nothing completes
+  int stream;              // 1: a CTA pairs its heads' Q tiles across head boundaries
+                           // (whole heads with an odd tile count), K/V streamed
 };
 
 template <int D>
@@ -212,30 +224,93 @@ __device__ __forceinline__ int block_cols(int N, int j) {
   return n16 < BK ? n16 : BK;
 }
 
-// One (unit, round) step of the schedule, identical for every role.
+// One round of the schedule (up to two Q tiles, one per slot), identical for
+// every role.  Both slots belong to one head except in stream mode.
 struct Round {
-  int b, h, r;  // image, head, round index within the head (tile index for tile units)
-  int t0;       // Q tile of slot 0 (slot 1 has t0 + 1)
-  int nslots;   // 2 = full round (tiles 2r, 2r+1), 1 = half round or a tile unit
-  bool first;   // first round of its unit
-  bool last;    // last round of its unit
+  int b0, b1, h0, h1, t0, t1;  // image, head and Q tile of slot 0 / slot 1
+  int nslots;                  // 2 = both slots, 1 = slot 0 only
+  bool shared_kv;              // both slots read one head's K/V: one K/V event per key block
+  bool first;                  // first round of its unit
+  bool last;                   // last round of its unit
+  // Per-slot fields by selects (no runtime-indexed arrays, which would live
+  // in local memory).
+  __device__ __forceinline__ int b(int s) const { return s ? b1 : b0; }
+  __device__ __forceinline__ int h(int s) const { return s ? h1 : h0; }
+  __device__ __forceinline__ int tile(int s) const { return s ? t1 : t0; }
 };
 
-__device__ __forceinline__ Round make_round(const AttnParams& p, int u, int rr) {
+// Walks this CTA's rounds: whole units (u strided by the grid, rounds rr of
+// each), or in stream mode the Q tiles of its heads two at a time.
+struct Cursor {
+  int u, rr;      // unit and round within it
+  int tq;         // stream mode: tile of head u for slot 0 of the next round
+};
+
+__device__ __forceinline__ Cursor cursor_start() {
+  return Cursor{static_cast<int>(blockIdx.x), 0, 0};
+}
+
+__device__ __forceinline__ bool cursor_more(const AttnParams& p, const Cursor& c) {
+  return c.u < p.num_units;
+}
+
+__device__ __forceinline__ Round next_round(const AttnParams& p, Cursor& c) {
   Round x;
-  const int bh = u / p.units_per_head;
-  x.r = (u % p.units_per_head) * p.rounds_per_unit + rr;
-  x.b = bh / p.H;
-  x.h = bh % p.H;
+  if (p.stream) {
+    // Slot 0: tile tq of head u; slot 1: the next tile, possibly of the next head.
+    int ub = c.u, tb = c.tq + 1;
+    if (tb == p.num_qtiles) {
+      ub = c.u + static_cast<int>(gridDim.x);
+      tb = 0;
+    }
+    x.nslots = ub < p.num_units ? 2 : 1;
+    if (x.nslots == 1) {
+      ub = c.u;
+      tb = c.tq;
+    }
+    x.b0 = c.u / p.H;
+    x.h0 = c.u - x.b0 * p.H;
+    x.t0 = c.tq;
+    if (ub == c.u) {
+      x.b1 = x.b0;
+      x.h1 = x.h0;
+    } else {
+      x.b1 = ub / p.H;
+      x.h1 = ub - x.b1 * p.H;
+    }
+    x.t1 = tb;
+    x.shared_kv = ub == c.u;
+    x.first = x.last = true;
+    // Advance two tiles.
+    c.u = ub;
+    c.tq = tb + 1;
+    if (x.nslots == 1 || c.tq == p.num_qtiles) {
+      c.u = x.nslots == 1 ? p.num_units : ub + static_cast<int>(gridDim.x);
+      c.tq = 0;
+    }
+    return x;
+  }
+  const int bh = c.u / p.units_per_head;
+  const int r = (c.u - bh * p.units_per_head) * p.rounds_per_unit + c.rr;
+  int t0;
   if (p.tile_units) {
-    x.t0 = x.r;
+    t0 = r;
     x.nslots = 1;
   } else {
-    x.t0 = 2 * x.r;
-    x.nslots = (2 * x.r + 1 < p.num_qtiles) ? 2 : 1;
+    t0 = 2 * r;
+    x.nslots = (2 * r + 1 < p.num_qtiles) ? 2 : 1;
   }
-  x.first = rr == 0;
-  x.last = rr == p.rounds_per_unit - 1;
+  x.b0 = x.b1 = bh / p.H;
+  x.h0 = x.h1 = bh - x.b0 * p.H;
+  x.t0 = t0;
+  x.t1 = t0 + 1;
+  x.shared_kv = true;
+  x.first = c.rr == 0;
+  x.last = c.rr == p.rounds_per_unit - 1;
+  if (++c.rr == p.rounds_per_unit) {
+    c.rr = 0;
+    c.u += static_cast<int>(gridDim.x);
+  }
   return x;
 }
 
@@ -271,51 +346,56 @@ __device__ void load_role(const AttnParams& p, uint32_t sQ, uint32_t sK, uint32_
       return false;
     if (elect_one()) {
       const uint32_t dst = sQ + s * G::kQBytes;
-      const int row0 = (x.t0 + s) * kQRows;
+      const int row0 = x.tile(s) * kQRows;
       mbar_arrive_expect_tx(bar.q_full(s), G::kQBytes);
-      tma_load_5d(dst, &p.tm_q, bar.q_full(s), 0, x.h, 0, row0, x.b);
+      tma_load_5d(dst, &p.tm_q, bar.q_full(s), 0, x.h(s), 0, row0, x.b(s));
       if (G::kHasTail)
-        tma_load_5d(dst + G::kQTail, &p.tm_q_tail, bar.q_full(s), 64, x.h, 0, row0, x.b);
+        tma_load_5d(dst + G::kQTail, &p.tm_q_tail, bar.q_full(s), 64, x.h(s), 0, row0, x.b(s));
     }
     __syncwarp();
     if (s == 0) ++nq0; else ++nq1;
     return true;
   };
-  auto load_kv = [&](uint32_t dst, uint32_t mbar, int w, int j, const Round& x) {
+  auto load_kv = [&](uint32_t dst, uint32_t mbar, int w, int j, int b, int hh) {
     if (elect_one()) {
       mbar_arrive_expect_tx(mbar, G::kKVBytes);
-      tma_load_5d(dst, &p.tm_kv, mbar, 0, x.h, w, j * G::BK, x.b);
+      tma_load_5d(dst, &p.tm_kv, mbar, 0, hh, w, j * G::BK, b);
       if (G::kHasTail)
-        tma_load_5d(dst + G::kKVTail, &p.tm_kv_tail, mbar, 64, x.h, w, j * G::BK, x.b);
+        tma_load_5d(dst + G::kKVTail, &p.tm_kv_tail, mbar, 64, hh, w, j * G::BK, b);
     }
     __syncwarp();
   };
 
-  for (int u = blockIdx.x; ok && u < p.num_units; u += gridDim.x) {
-    for (int rr = 0; ok && rr < p.rounds_per_unit; ++rr) {
-      const Round x = make_round(p, u, rr);
-      if (!p.reuse || x.first) {
-        for (int j = 0; ok && j < nb; ++j) {
-          const int slot = pos.slot;
-          if (!wait_bounded(bar.k_empty(slot), pos.phase ^ 1u, abort_flag, p.wait_limit_ns,
-                            kSiteLoadK) ||
-              !wait_bounded(bar.v_empty(slot), pos.phase ^ 1u, abort_flag, p.wait_limit_ns,
-                            kSiteLoadV)) {
-            ok = false;
-            break;
-          }
-          load_kv(sK + slot * G::kKVStride, bar.k_full(slot), 1, j, x);
-          if (j == 0) {
-            // Q tiles right after the first K block so S(0) can start early.
-            for (int s = 0; ok && s < x.nslots; ++s) ok = load_q(s, x);
-          }
-          load_kv(sV + slot * G::kKVStride, bar.v_full(slot), 2, j, x);
-          ++kv_ev;
-          pos.advance(R);
+  for (Cursor cu = cursor_start(); ok && cursor_more(p, cu);) {
+    const Round x = next_round(p, cu);
+    if (!p.reuse || x.first) {
+      const int E = x.shared_kv ? nb : 2 * nb;
+      for (int e = 0; ok && e < E; ++e) {
+        const int se = x.shared_kv ? 0 : (e & 1);
+        const int j = x.shared_kv ? e : (e >> 1);
+        const int slot = pos.slot;
+        if (!wait_bounded(bar.k_empty(slot), pos.phase ^ 1u, abort_flag, p.wait_limit_ns,
+                          kSiteLoadK) ||
+            !wait_bounded(bar.v_empty(slot), pos.phase ^ 1u, abort_flag, p.wait_limit_ns,
+                          kSiteLoadV)) {
+          ok = false;
+          break;
         }
-      } else {
-        for (int s = 0; ok && s < x.nslots; ++s) ok = load_q(s, x);
+        load_kv(sK + slot * G::kKVStride, bar.k_full(slot), 1, j, x.b(se), x.h(se));
+        if (j == 0) {
+          // Q tiles right after their first K block so S(0) can start early.
+          if (x.shared_kv) {
+            for (int s = 0; ok && s < x.nslots; ++s) ok = load_q(s, x);
+          } else {
+            ok = load_q(se, x);
+          }
+        }
+        load_kv(sV + slot * G::kKVStride, bar.v_full(slot), 2, j, x.b(se), x.h(se));
+        ++kv_ev;
+        pos.advance(R);
       }
+    } else {
+      for (int s = 0; ok && s < x.nslots; ++s) ok = load_q(s, x);
     }
   }
   // Wait (bounded) until every copy this thread issued has landed.
@@ -441,56 +521,57 @@ __device__ void mma_role(const AttnParams& p, uint32_t tmem, uint32_t sQ, uint32
   };
 
   bool ok = true;
-  for (int u = blockIdx.x; ok && u < p.num_units; u += gridDim.x) {
-    const RingPos unit_pos = pos;
-    for (int rr = 0; ok && rr < p.rounds_per_unit; ++rr) {
-      const Round x = make_round(p, u, rr);
-      const int ns = x.nslots;
-      const bool release = !p.reuse || x.last;
-      RingPos cur = p.reuse ? unit_pos : pos;  // K/V event of key block j
-      if (score_warp) {
-        // S of the first key block for every slot (the previous round's last
-        // S of each slot was read out before its s_free phase was consumed).
-        if (!(ok = wait_k(cur))) break;
+  RingPos unit_pos = pos;
+  for (Cursor cu = cursor_start(); ok && cursor_more(p, cu);) {
+    const Round x = next_round(p, cu);
+    if (x.first) unit_pos = pos;
+    const int ns = x.nslots;
+    const bool sh = x.shared_kv;
+    const bool release = !p.reuse || x.last;
+    RingPos cur = p.reuse ? unit_pos : pos;  // K/V event of the next (block, slot)
+    if (score_warp) {
+      // S of block j for slot s as soon as slot s has read S of block j-1.
+      for (int j = 0; ok && j < nb; ++j) {
         for (int s = 0; ok && s < ns; ++s) {
-          if (!(ok = wait_q(s))) break;
-          scores(s, 0, cur.slot);
-          if (nb == 1) commit(bar.q_empty(s));
+          if ((!sh || s == 0) && !(ok = wait_k(cur))) break;
+          if (!(ok = (j == 0 ? wait_q(s) : wait_free(s)))) break;
+          scores(s, j, cur.slot);
+          if (j == nb - 1) commit(bar.q_empty(s));
+          if (!sh) {
+            if (release) commit(bar.k_empty(cur.slot));
+            cur.advance(R);
+          }
         }
         if (!ok) break;
-        if (release) commit(bar.k_empty(cur.slot));
-        // S of block j+1 for slot s as soon as slot s has read S of block j.
-        for (int j = 0; ok && j + 1 < nb; ++j) {
-          cur.advance(R);
-          if (!(ok = wait_k(cur))) break;
-          for (int s = 0; s < ns; ++s) {
-            if (!(ok = wait_free(s))) break;
-            scores(s, j + 1, cur.slot);
-            if (j + 1 == nb - 1) commit(bar.q_empty(s));
-          }
-          if (!ok) break;
+        if (sh) {
           if (release) commit(bar.k_empty(cur.slot));
+          cur.advance(R);
+        }
+      }
+      if (!ok) break;
+      for (int s = 0; ok && s < ns; ++s) ok = wait_free(s);  // last block read out
+      if (!ok) break;
+    } else {
+      // P V of block j for slot s as soon as slot s has stored P of block j.
+      for (int j = 0; ok && j < nb; ++j) {
+        for (int s = 0; ok && s < ns; ++s) {
+          if ((!sh || s == 0) && !(ok = wait_v(cur))) break;
+          if (!(ok = wait_p(s))) break;
+          values(s, j, cur.slot);
+          if (!sh) {
+            if (release) commit(bar.v_empty(cur.slot));
+            cur.advance(R);
+          }
         }
         if (!ok) break;
-        for (int s = 0; ok && s < ns; ++s) ok = wait_free(s);  // last block read out
-        if (!ok) break;
-        cur.advance(R);
-      } else {
-        // P V of block j for slot s as soon as slot s has stored P of block j.
-        for (int j = 0; ok && j < nb; ++j) {
-          if (!(ok = wait_v(cur))) break;
-          for (int s = 0; s < ns; ++s) {
-            if (!(ok = wait_p(s))) break;
-            values(s, j, cur.slot);
-          }
-          if (!ok) break;
+        if (sh) {
           if (release) commit(bar.v_empty(cur.slot));
           cur.advance(R);
         }
-        if (!ok) break;
       }
-      pos = cur;  // first event after this round (reuse: after the unit)
+      if (!ok) break;
     }
+    pos = cur;  // first event after this round (reuse: after the unit)
   }
   // Every tensor-core operation this warp issued must finish before the
   // tensor memory is freed.
@@ -651,59 +732,57 @@ __device__ void softmax_role(const AttnParams& p, uint32_t tmem, const Barriers&
     return;
   }
 
-  for (int u = blockIdx.x; u < p.num_units; u += gridDim.x) {
-    for (int rr = 0; rr < p.rounds_per_unit; ++rr) {
-      const Round x = make_round(p, u, rr);
-      const bool full = x.nslots == 2;
-      if (!full && s == 1) continue;
-      const int tile = x.t0 + s;
-      SoftState st{-INFINITY, 0.0f};
-      for (int j = 0; j < nb; ++j) {
-        if (!wait_bounded(bar.s_full(s), ns & 1u, abort_flag, p.wait_limit_ns, kSiteSoftS))
-          return;
-        ++ns;
-        tc_fence_after();
-        VLA_TRACE_EVENT(kTrSoftS, s, j);
-        const bool ok = softmax_block_dispatch<D>(
-            p, st, tS, tO, tP, block_cols<G::BK>(p.N, j), min(G::BK, p.N - j * G::BK), j, bar, s,
-            (npv + j - 1) & 1u, abort_flag, lane);
-        if (!ok) return;
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(bar.p_full(s));
-        VLA_TRACE_EVENT(kTrSoftP, s, j);
-      }
-      // Epilogue: wait for the last P V, then O / l -> bf16, 16-byte stores.
-      if (!wait_bounded(bar.o_prog(s), (npv + nb - 1) & 1u, abort_flag, p.wait_limit_ns,
-                        kSiteSoftO))
+  for (Cursor cu = cursor_start(); cursor_more(p, cu);) {
+    const Round x = next_round(p, cu);
+    const bool full = x.nslots == 2;
+    if (!full && s == 1) continue;
+    const int tile = x.tile(s);
+    SoftState st{-INFINITY, 0.0f};
+    for (int j = 0; j < nb; ++j) {
+      if (!wait_bounded(bar.s_full(s), ns & 1u, abort_flag, p.wait_limit_ns, kSiteSoftS))
         return;
-      npv += nb;
+      ++ns;
       tc_fence_after();
-      VLA_TRACE_EVENT(kTrSoftEpi, s, 0);
-      const float inv_l = 1.0f / st.l_run;
-      uint32_t ob[64];
-      tmem_ld64(tO, ob);
-      uint32_t ot[16];
-      if (G::DP > 64) tmem_ld16(tO + 64, ot);
-      const int row = tile * kQRows + row_in_tile;
-      if (row < p.N) {
-        uint4* dst = reinterpret_cast<uint4*>(
-            p.o + ((static_cast<size_t>(x.b) * p.N + row) * p.H + x.h) * D);
+      VLA_TRACE_EVENT(kTrSoftS, s, j);
+      const bool ok = softmax_block_dispatch<D>(
+          p, st, tS, tO, tP, block_cols<G::BK>(p.N, j), min(G::BK, p.N - j * G::BK), j, bar, s,
+          (npv + j - 1) & 1u, abort_flag, lane);
+      if (!ok) return;
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar.p_full(s));
+      VLA_TRACE_EVENT(kTrSoftP, s, j);
+    }
+    // Epilogue: wait for the last P V, then O / l -> bf16, 16-byte stores.
+    if (!wait_bounded(bar.o_prog(s), (npv + nb - 1) & 1u, abort_flag, p.wait_limit_ns,
+                      kSiteSoftO))
+      return;
+    npv += nb;
+    tc_fence_after();
+    VLA_TRACE_EVENT(kTrSoftEpi, s, 0);
+    const float inv_l = 1.0f / st.l_run;
+    uint32_t ob[64];
+    tmem_ld64(tO, ob);
+    uint32_t ot[16];
+    if (G::DP > 64) tmem_ld16(tO + 64, ot);
+    const int row = tile * kQRows + row_in_tile;
+    if (row < p.N) {
+      uint4* dst = reinterpret_cast<uint4*>(
+          p.o + ((static_cast<size_t>(x.b(s)) * p.N + row) * p.H + x.h(s)) * D);
 #pragma unroll
-        for (int t = 0; t < D / 8; ++t) {
-          float v[8];
+      for (int t = 0; t < D / 8; ++t) {
+        float v[8];
 #pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            const int ch = 8 * t + e;
-            v[e] = __uint_as_float(ch < 64 ? ob[ch] : ot[ch - 64]) * inv_l;
-          }
-          uint4 w;
-          w.x = pack_bf16x2(v[0], v[1]);
-          w.y = pack_bf16x2(v[2], v[3]);
-          w.z = pack_bf16x2(v[4], v[5]);
-          w.w = pack_bf16x2(v[6], v[7]);
-          dst[t] = w;
+        for (int e = 0; e < 8; ++e) {
+          const int ch = 8 * t + e;
+          v[e] = __uint_as_float(ch < 64 ? ob[ch] : ot[ch - 64]) * inv_l;
         }
+        uint4 w;
+        w.x = pack_bf16x2(v[0], v[1]);
+        w.y = pack_bf16x2(v[2], v[3]);
+        w.z = pack_bf16x2(v[4], v[5]);
+        w.w = pack_bf16x2(v[6], v[7]);
+        dst[t] = w;
       }
     }
   }

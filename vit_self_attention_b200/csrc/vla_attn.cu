@@ -209,16 +209,19 @@ int launch(const void* q, void* o, int B, int N, int H, float scale, cudaStream_
   // Work units: whole heads (K/V loaded once per head) when there are enough
   // heads to fill the SMs; otherwise single Q tiles if all of them fit on the
   // SMs at once (shortest per-CTA chain), else single rounds of two tiles.
+  // Whole heads with an odd tile count run in stream mode: the CTA pairs its
+  // heads' tiles across head boundaries (no half rounds) and streams K/V.
   prm.rounds_per_head = (nq + 1) / 2;
   const long long heads = static_cast<long long>(B) * H;
   prm.rounds_per_unit = heads >= di.sm_count ? prm.rounds_per_head : 1;
   prm.tile_units = (heads < di.sm_count && nq > 1 && heads * nq <= di.sm_count) ? 1 : 0;
+  prm.stream = (heads >= di.sm_count && nq > 1 && (nq & 1)) ? 1 : 0;
   prm.units_per_head = prm.tile_units ? nq : prm.rounds_per_head / prm.rounds_per_unit;
   const long long units = heads * prm.units_per_head;
   if (units > 0x7FFFFFFFll) return VLA_ATTN_ERR_SHAPE;
   prm.num_units = static_cast<int>(units);
   prm.ring = ring;
-  prm.reuse = nb <= ring ? 1 : 0;
+  prm.reuse = (nb <= ring && !prm.stream) ? 1 : 0;
   prm.c = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
   const unsigned long long lim = g_wait_limit_ns.load();
   prm.wait_limit_ns = lim == 0 ? kDefaultWaitLimitNs : lim;
