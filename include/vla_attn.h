@@ -87,11 +87,19 @@ int vla_attn_fwd(const void* q, const void* k, const void* v, void* o,
  * End-to-end variant for callers whose data live in host memory: copies the
  * packed [B, N, 3, H, d] bf16 input from `qkv_host` into the caller's device
  * buffer `qkv_dev`, runs vla_attn_fwd on it into `o_dev`, and copies the
- * [B, N, H, d] bf16 result back to `o_host` -- all enqueued on `stream`, one
- * cudaMemcpyAsync per direction.  Host buffers should be pinned
- * (cudaHostAlloc / cudaHostRegister) for the copies to be asynchronous.  The
- * host result is valid once the stream has been synchronised.  Same argument
- * rules and status codes as vla_attn_fwd; allocates nothing.
+ * [B, N, H, d] bf16 result back to `o_host`.  A batch of at least two chunks
+ * (a chunk = the fewest whole images with 4 heads per SM) is pipelined per
+ * chunk: input copy and kernel on `stream`, result copy on an internal
+ * copy-out stream of the device, so that it overlaps the next chunk's input
+ * copy; `stream` then waits for the copy-out stream.  Smaller batches use one
+ * copy per direction on `stream`.  Either way the results are those of
+ * vla_attn_fwd on the whole batch, and the host result is valid once
+ * `stream` has been synchronised.  Host buffers should be pinned
+ * (cudaHostAlloc / cudaHostRegister) for the copies to be asynchronous.
+ * Same argument rules and status codes as vla_attn_fwd.  Allocates no memory;
+ * the first pipelined call on a device creates the copy-out stream and two
+ * events, which live as long as the process.  Calls are serialised on a
+ * library lock while they enqueue.
  */
 int vla_attn_fwd_host(const void* qkv_host, void* o_host, void* qkv_dev, void* o_dev,
                       int B, int N, int H, int d, float scale, void* stream);

@@ -202,6 +202,31 @@ def test_host_buffer_entry():
     assert_parity(got, want, "host-buffer entry")
 
 
+def test_host_buffer_entry_pipelined_chunks():
+    """A batch of several chunks takes the pipelined host path (copy-out stream): the
+    host result equals the device entry's bytes, on two calls in a row."""
+    import vit_self_attention_b200 as vab
+    sm = torch.cuda.get_device_properties(0).multi_processor_count
+    H, N, d = 16, 197, 64
+    chunk = -(-4 * sm // H)
+    B = 2 * chunk + 3  # two full chunks and a ragged one
+    bits = si.packed_qkv(B, N, H, d, seed=4242)
+    scale = 1.0 / math.sqrt(d)
+    host_in = torch.from_numpy(bits.view(np.int16).copy()).pin_memory()
+    dev_in = torch.empty(bits.shape, dtype=torch.int16, device="cuda")
+    dev_out = torch.empty((B, N, H, d), dtype=torch.int16, device="cuda")
+    ref = vab.attention(host_in.cuda().view(torch.bfloat16), scale).view(torch.int16).cpu()
+    for _ in range(2):
+        host_out = torch.full((B, N, H, d), -1, dtype=torch.int16).pin_memory()
+        vab.vla_attn_fwd_host(host_in, host_out, dev_in, dev_out, B, N, H, d, scale)
+        torch.cuda.current_stream().synchronize()
+        assert torch.equal(host_out, ref)
+    rows = [(0, 0, 0), (chunk, 5, 196), (B - 1, 15, 100)]
+    got = si.bf16_bits_to_f32(host_out.numpy().view(np.uint16)).astype(np.float64)
+    want = oracle.attention_rows_packed_bf16(bits, scale, rows)
+    assert_parity(np.stack([got[b, n, h] for b, h, n in rows]), want, "pipelined host entry")
+
+
 def test_device_status_clean_and_launch_count():
     import vit_self_attention_b200 as vab
     n0 = vab.vla_attn_launch_count()

@@ -85,6 +85,39 @@ int device_info(int dev, DeviceInfo* out) {
   return di.supported ? VLA_ATTN_OK : VLA_ATTN_ERR_DEVICE;
 }
 
+// Copy-out stream and fork / join events of the pipelined host-buffer entry,
+// one set per device, created on first use (guarded by g_pipe_mutex, which
+// the caller holds for the whole enqueue sequence).
+struct HostPipe {
+  cudaStream_t out = nullptr;
+  cudaEvent_t fork = nullptr;
+  cudaEvent_t join = nullptr;
+};
+
+std::mutex g_pipe_mutex;
+HostPipe g_pipe[kMaxDevices];
+
+int host_pipe(int dev, HostPipe** out) {
+  HostPipe& p = g_pipe[dev];
+  if (p.out == nullptr) {
+    cudaStream_t s = nullptr;
+    cudaEvent_t f = nullptr, j = nullptr;
+    if (cudaStreamCreateWithFlags(&s, cudaStreamNonBlocking) != cudaSuccess)
+      return VLA_ATTN_ERR_CUDA;
+    if (cudaEventCreateWithFlags(&f, cudaEventDisableTiming) != cudaSuccess ||
+        cudaEventCreateWithFlags(&j, cudaEventDisableTiming) != cudaSuccess) {
+      if (f != nullptr) cudaEventDestroy(f);
+      cudaStreamDestroy(s);
+      return VLA_ATTN_ERR_CUDA;
+    }
+    p.out = s;
+    p.fork = f;
+    p.join = j;
+  }
+  *out = &p;
+  return VLA_ATTN_OK;
+}
+
 // Raises the kernel's dynamic shared-memory limit to at least `smem` bytes.
 template <int D>
 int ensure_smem_attr(int dev, int smem) {
@@ -282,16 +315,66 @@ int vla_attn_fwd_host(const void* qkv_host, void* o_host, void* qkv_dev, void* o
   const size_t hd_bytes = static_cast<size_t>(H > 0 ? H : 0) * (d > 0 ? d : 0) * 2u;
   int rc = check_args(qd, qd + hd_bytes, qd + 2 * hd_bytes, o_dev, B, N, H, d, scale);
   if (rc != VLA_ATTN_OK) return rc;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return VLA_ATTN_ERR_CUDA;
+  DeviceInfo di;
+  if ((rc = device_info(dev, &di)) != VLA_ATTN_OK) return rc;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  const size_t in_bytes = 3ull * B * N * H * d * 2ull;
-  const size_t out_bytes = 1ull * B * N * H * d * 2ull;
-  if (cudaMemcpyAsync(qkv_dev, qkv_host, in_bytes, cudaMemcpyHostToDevice, st) != cudaSuccess)
-    return VLA_ATTN_ERR_CUDA;
-  rc = vla_attn_fwd(qd, qd + hd_bytes, qd + 2 * hd_bytes, o_dev, B, N, H, d, scale, stream);
-  if (rc != VLA_ATTN_OK) return rc;
-  if (cudaMemcpyAsync(o_host, o_dev, out_bytes, cudaMemcpyDeviceToHost, st) != cudaSuccess)
-    return VLA_ATTN_ERR_CUDA;
-  return VLA_ATTN_OK;
+  const size_t img_out = static_cast<size_t>(N) * H * d * 2u;  // bytes of one image's O
+  const size_t img_in = 3u * img_out;                           // and of its packed QKV
+  // Chunks of whole images, each with at least 4 heads per SM so that every
+  // launch still fills the GPU; a batch smaller than two chunks goes in one.
+  const long long min_heads = 4ll * di.sm_count;
+  const int chunk = static_cast<int>((min_heads + H - 1) / H);
+  if (B < 2 * chunk) {
+    if (cudaMemcpyAsync(qkv_dev, qkv_host, img_in * B, cudaMemcpyHostToDevice, st) != cudaSuccess)
+      return VLA_ATTN_ERR_CUDA;
+    rc = vla_attn_fwd(qd, qd + hd_bytes, qd + 2 * hd_bytes, o_dev, B, N, H, d, scale, stream);
+    if (rc != VLA_ATTN_OK) return rc;
+    if (cudaMemcpyAsync(o_host, o_dev, img_out * B, cudaMemcpyDeviceToHost, st) != cudaSuccess)
+      return VLA_ATTN_ERR_CUDA;
+    return VLA_ATTN_OK;
+  }
+  // Pipelined: chunk i's host-to-device copy and kernel on `stream`, its
+  // device-to-host copy on the device's copy-out stream, so it overlaps the
+  // next chunk's host-to-device copy (the two directions use separate copy
+  // engines).  `stream` waits for the copy-out stream at the end.
+  std::lock_guard<std::mutex> lock(g_pipe_mutex);
+  HostPipe* pipe = nullptr;
+  if ((rc = host_pipe(dev, &pipe)) != VLA_ATTN_OK) return rc;
+  const char* hin = static_cast<const char*>(qkv_host);
+  char* hout = static_cast<char*>(o_host);
+  char* din = static_cast<char*>(qkv_dev);
+  char* dout = static_cast<char*>(o_dev);
+  bool forked = false;
+  for (int b0 = 0; b0 < B && rc == VLA_ATTN_OK; b0 += chunk) {
+    const int nbi = B - b0 < chunk ? B - b0 : chunk;
+    const size_t in_off = img_in * b0, out_off = img_out * b0;
+    if (cudaMemcpyAsync(din + in_off, hin + in_off, img_in * nbi, cudaMemcpyHostToDevice, st) !=
+        cudaSuccess) {
+      rc = VLA_ATTN_ERR_CUDA;
+      break;
+    }
+    const char* q = din + in_off;
+    rc = vla_attn_fwd(q, q + hd_bytes, q + 2 * hd_bytes, dout + out_off, nbi, N, H, d, scale,
+                      stream);
+    if (rc != VLA_ATTN_OK) break;
+    if (cudaEventRecord(pipe->fork, st) != cudaSuccess ||
+        cudaStreamWaitEvent(pipe->out, pipe->fork, 0) != cudaSuccess) {
+      rc = VLA_ATTN_ERR_CUDA;
+      break;
+    }
+    forked = true;
+    if (cudaMemcpyAsync(hout + out_off, dout + out_off, img_out * nbi, cudaMemcpyDeviceToHost,
+                        pipe->out) != cudaSuccess)
+      rc = VLA_ATTN_ERR_CUDA;
+  }
+  // Join even after an error, so that work already on the copy-out stream is
+  // ordered before anything later on `stream`.
+  if (forked && (cudaEventRecord(pipe->join, pipe->out) != cudaSuccess ||
+                 cudaStreamWaitEvent(st, pipe->join, 0) != cudaSuccess))
+    rc = VLA_ATTN_ERR_CUDA;
+  return rc;
 }
 
 const char* vla_attn_strerror(int status) {
@@ -302,7 +385,7 @@ const char* vla_attn_strerror(int status) {
       return "bad shape: B, N, H must be >= 1 and q/k/v must point into one packed [B,N,3,H,d] "
              "buffer (k = q + H*d, v = q + 2*H*d elements)";
     case VLA_ATTN_ERR_UNSUPPORTED:
-      return "unsupported: head dimension must be 64 or 72 and N at most 577";
+      return "unsupported: head dimension must be 64 or 72 and N at most vla_attn_max_tokens(d)";
     case VLA_ATTN_ERR_ALIGN: return "q and o must be 16-byte aligned";
     case VLA_ATTN_ERR_SCALE: return "scale must be finite and > 0";
     case VLA_ATTN_ERR_CUDA: return "a CUDA runtime or driver call failed";
