@@ -36,7 +36,7 @@ if ROOT not in sys.path:
 
 import seeded_inputs as si  # noqa: E402
 
-WORKLOAD = si.CONFIGS[4]  # vit_l14_336px_b256
+WORKLOAD = si.VIT_L14_336PX_B256
 METRIC = "attention TFLOP/s (4*B*H*N^2*d per call) on B200"
 UNIT = "TFLOP/s"
 KERNEL_SOURCES = ["vit_self_attention_b200/csrc/attn_kernel.cuh",
@@ -391,7 +391,7 @@ def run_configs(args) -> None:
             ts.append(e0.elapsed_time(e1) * 1e3)  # us
         return ts
 
-    items = [(c, True) for c in si.CONFIGS] + [
+    items = [(c, True) for c in si.WORKLOADS] + [
         (si.AttnConfig(6, "vit_l14_384px_b64", 64, 730, 16, 64, 0.125, 1.0, 1.0, 1, 24), False),
         (si.AttnConfig(7, "vit_l14_448px_b64", 64, 1025, 16, 64, 0.125, 1.0, 1.0, 1, 24), False)]
     for c, std in items:
@@ -554,7 +554,7 @@ def run_block(args) -> None:
                 "w1": t_((F, W), 0.0, 1.0 / _m.sqrt(W), seed + 8), "b1": t_((F,), 0.0, 0.1, seed + 9),
                 "w2": t_((W, F), 0.0, 1.0 / _m.sqrt(F), seed + 10), "b2": t_((W,), 0.0, 0.1, seed + 11)}
 
-    for c in list(si.CONFIGS[1:4]) + [si.CONFIGS[4]]:
+    for c in list(si.ENCODER_WORKLOADS[1:]) + [si.VIT_L14_336PX_B256]:
         W = c.H * c.d
         F = mlp_width[W]
         M = c.B * c.N

@@ -39,8 +39,14 @@ _TWO_M53 = 2.0 ** -53
 
 __all__ = [
     "AttnConfig",
-    "CONFIGS",
-    "config_by_name",
+    "WORKLOADS",
+    "ENCODER_WORKLOADS",
+    "VIT_B16_112PX_1VIEW",
+    "VIT_B16_224PX_3VIEWS",
+    "VIT_L14_224PX_3VIEWS",
+    "SIGLIP_SO400M14_224PX_2VIEWS",
+    "VIT_L14_336PX_B256",
+    "workload",
     "call_seed",
     "splitmix64_draws",
     "normals",
@@ -175,7 +181,7 @@ def call_seed(config_index: int, call: int) -> int:
     return 1000 * config_index + call
 
 
-CONFIGS = (
+WORKLOADS = (
     # ViT-B/16 at 112x112, one camera view: 49 patches + CLS.
     AttnConfig(1, "vit_b16_112px_1view", 1, 50, 12, 64, 1.0 / 8.0, 1.0, 1.0, 1, 12),
     # ViT-B/16 at 224x224, three camera views (Main/Side/Top), 12 layers.
@@ -191,8 +197,15 @@ CONFIGS = (
 )
 
 
-def config_by_name(name: str) -> AttnConfig:
-    for c in CONFIGS:
-        if c.name == name or str(c.index) == str(name):
+(VIT_B16_112PX_1VIEW, VIT_B16_224PX_3VIEWS, VIT_L14_224PX_3VIEWS, SIGLIP_SO400M14_224PX_2VIEWS,
+ VIT_L14_336PX_B256) = WORKLOADS
+# The camera-view encoder workloads (µs-scale calls, many layers per image batch).
+ENCODER_WORKLOADS = WORKLOADS[:4]
+
+
+def workload(name: str) -> AttnConfig:
+    """The workload with this name (``vit_l14_336px_b256`` and so on)."""
+    for c in WORKLOADS:
+        if c.name == name:
             return c
     raise KeyError(name)

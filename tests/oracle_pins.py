@@ -201,24 +201,24 @@ def _widen(bits):
     return si.bf16_bits_to_f32(bits).astype(np.float64)
 
 
-def pin_torch_sdpa_configs(lib, configs=(1, 2, 3, 4)):
-    """PyTorch's CPU scaled_dot_product_attention in fp64 on the seeded config inputs,
-    sliced from the packed buffer by numpy (independently of the oracle's own slicing)."""
-    for ci in configs:
-        c = si.CONFIGS[ci - 1]
+def pin_torch_sdpa_workloads(lib, workloads=si.ENCODER_WORKLOADS):
+    """PyTorch's CPU scaled_dot_product_attention in fp64 on the seeded encoder workload
+    inputs, sliced from the packed buffer by numpy (independently of the oracle's own
+    slicing)."""
+    for c in workloads:
         bits = c.qkv(0)
         x = _widen(bits)
         q, k, v = x[:, :, 0], x[:, :, 1], x[:, :, 2]
         want = _torch_sdpa(q, k, v, c.scale)
         got = lib.attention_packed_bf16(bits, c.scale)
-        _close(got, want, 1e-12, f"config {ci} vs torch SDPA fp64")
+        _close(got, want, 1e-12, f"{c.name} vs torch SDPA fp64")
         got2 = lib.attention_f64(q, k, v, c.scale)
-        _close(got2, want, 1e-12, f"config {ci} fp64 entry vs torch SDPA fp64")
+        _close(got2, want, 1e-12, f"{c.name} fp64 entry vs torch SDPA fp64")
 
 
 def pin_torch_sdpa_large_slice(lib):
     """One image of the 336px ViT-L/14 shape (N = 577, H = 16, d = 64) against torch SDPA."""
-    c = si.CONFIGS[4]
+    c = si.VIT_L14_336PX_B256
     bits = si.packed_qkv(1, c.N, c.H, c.d, c.seed(0))
     x = _widen(bits)
     want = _torch_sdpa(x[:, :, 0], x[:, :, 1], x[:, :, 2], c.scale)
@@ -242,7 +242,7 @@ def pin_d72_zero_padding(lib):
 
 def pin_rows_entry(lib):
     """The sampled-rows entry returns exactly the full computation's rows."""
-    c = si.CONFIGS[2]
+    c = si.VIT_L14_224PX_3VIEWS
     bits = c.qkv(3)
     full = lib.attention_packed_bf16(bits, c.scale)
     rows = [(0, 0, 0), (2, 15, 256), (1, 7, 128), (2, 3, 1)]
@@ -517,7 +517,7 @@ ALL_PINS = [
     pin_head_batch_independence,
     pin_hard_attention,
     pin_brute_force_python,
-    pin_torch_sdpa_configs,
+    pin_torch_sdpa_workloads,
     pin_d72_zero_padding,
     pin_rows_entry,
     pin_layernorm_closed_forms,

@@ -25,11 +25,11 @@ pytestmark = [pytest.mark.gpu, needs_gpu]
 KNOWN_SITES = {1, 2, 3, 11, 12, 13, 14, 15, 21, 22, 31, 41}
 
 
-@pytest.mark.parametrize("cfg", [1, 3])
-def test_bounded_wait_runs_out_and_context_recovers(cfg):
+@pytest.mark.parametrize("name", ["vit_b16_224px_3views", "siglip_so400m14_224px_2views"])
+def test_bounded_wait_runs_out_and_context_recovers(name):
     import vit_self_attention_b200 as vab
 
-    c = si.CONFIGS[cfg]
+    c = si.workload(name)
     bits = c.qkv(0)
     vab.vla_attn_reset_device_status()
     vab.vla_attn_set_wait_limit_ns(2_000_000)
@@ -47,6 +47,6 @@ def test_bounded_wait_runs_out_and_context_recovers(cfg):
 
     # The context is usable and a normal call gives the right answer.
     got = run_cuda(bits, c.scale)
-    assert_parity(got, oracle.attention_packed_bf16(bits, c.scale), f"after abort, cfg{cfg + 1}")
+    assert_parity(got, oracle.attention_packed_bf16(bits, c.scale), f"after abort, {name}")
     st, site = vab.vla_attn_last_device_status()
     assert (st, site) == (0, 0)

@@ -27,7 +27,7 @@ from gpu_helpers import assert_close_bf16, assert_parity, needs_gpu
 pytestmark = [pytest.mark.gpu, needs_gpu]
 
 # (name, B, N, H, d): the encoder workloads; width W = H d, tokens M = B N.
-ENCODERS = [(c.name, c.B, c.N, c.H, c.d) for c in si.CONFIGS[:4]]
+ENCODERS = [(c.name, c.B, c.N, c.H, c.d) for c in si.ENCODER_WORKLOADS]
 
 
 def dev(bits):
@@ -129,12 +129,14 @@ def block_weights(W, seed):
             "bo": si.normal_bf16(seed + 5, (W,), 0.0, 0.1)}
 
 
-@pytest.mark.parametrize("cfg", [0, 1, 3])
-def test_attention_half_block_stagewise(cfg):
+@pytest.mark.parametrize("name", ["vit_b16_112px_1view", "vit_b16_224px_3views",
+                                  "siglip_so400m14_224px_2views"])
+def test_attention_half_block_stagewise(name):
     """x -> LayerNorm -> qkv linear -> attention -> output linear + residual x, each stage
     against the oracle on the GPU's own bf16 input to that stage."""
     import vit_self_attention_b200 as vab
-    c = si.CONFIGS[cfg]
+    c = si.workload(name)
+    cfg = c.index - 1  # seed offset of this workload
     W = c.H * c.d
     x = si.normal_bf16(700 + cfg, (c.B, c.N, W))
     p = block_weights(W, 710 + cfg)
@@ -159,7 +161,7 @@ def test_half_block_graph_capture():
     """Two layers of the chain captured in one CUDA graph and replayed give the same bytes
     as the eager calls."""
     import vit_self_attention_b200 as vab
-    c = si.CONFIGS[1]
+    c = si.VIT_B16_224PX_3VIEWS
     W = c.H * c.d
     x0 = dev(si.normal_bf16(800, (c.B, c.N, W)))
     layers = [{k: dev(v) for k, v in block_weights(W, 810 + 10 * i).items()} for i in range(2)]
@@ -266,12 +268,13 @@ def test_linear_gelu_variants(M, K, N, bias):
                       f"linear + GELU M={M} K={K} N={N} bias={bias}", mag=gelu_magnitude(x, w, b))
 
 
-def _layer_stagewise(cfg, fused_norm):
+def _layer_stagewise(name, fused_norm):
     """One pre-norm encoder layer on the GPU, each stage against the oracle on the GPU's
     own bf16 input to that stage.  fused_norm: the output projection leaves the residual
     to the fused add + LayerNorm; otherwise it adds it in its epilogue and LN2 is plain."""
     import vit_self_attention_b200 as vab
-    c = si.CONFIGS[cfg]
+    c = si.workload(name)
+    cfg = c.index - 1  # seed offset of this workload
     W = c.H * c.d
     F = MLP[W]
     x = si.normal_bf16(1300 + cfg, (c.B, c.N, W))
@@ -314,21 +317,22 @@ def _layer_stagewise(cfg, fused_norm):
                       mag=residual_magnitude(ab, p["w2"], p["b2"], hh))
 
 
-@pytest.mark.parametrize("cfg", [0, 1, 3])
-def test_encoder_layer_stagewise(cfg):
-    _layer_stagewise(cfg, fused_norm=False)
+@pytest.mark.parametrize("name", ["vit_b16_112px_1view", "vit_b16_224px_3views",
+                                  "siglip_so400m14_224px_2views"])
+def test_encoder_layer_stagewise(name):
+    _layer_stagewise(name, fused_norm=False)
 
 
-@pytest.mark.parametrize("cfg", [1, 3])
-def test_encoder_layer_stagewise_fused_residual_norm(cfg):
-    _layer_stagewise(cfg, fused_norm=True)
+@pytest.mark.parametrize("name", ["vit_b16_224px_3views", "siglip_so400m14_224px_2views"])
+def test_encoder_layer_stagewise_fused_residual_norm(name):
+    _layer_stagewise(name, fused_norm=True)
 
 
 def test_encoder_layers_graph_capture():
     """Two whole encoder layers captured in one CUDA graph and replayed give the eager
     bytes."""
     import vit_self_attention_b200 as vab
-    c = si.CONFIGS[3]
+    c = si.SIGLIP_SO400M14_224PX_2VIEWS
     W = c.H * c.d
     F = MLP[W]
     x0 = dev(si.normal_bf16(1400, (c.B, c.N, W)))

@@ -15,10 +15,9 @@ from gpu_helpers import assert_parity, device_qkv, needs_gpu, run_cuda
 pytestmark = [pytest.mark.gpu, needs_gpu]
 
 
-@pytest.mark.parametrize("cfg", [1, 2, 3, 4])
-def test_configs_every_call(cfg):
+@pytest.mark.parametrize("c", si.ENCODER_WORKLOADS, ids=lambda c: c.name)
+def test_encoder_workloads_every_call(c):
     """Every seeded layer call of the four encoder workloads."""
-    c = si.CONFIGS[cfg - 1]
     for call in range(c.calls):
         bits = c.qkv(call)
         want = oracle.attention_packed_bf16(bits, c.scale)
@@ -134,7 +133,7 @@ def test_large_config_sampled_rows_and_hull():
     configuration: complete heads and scattered rows against the oracle, and every
     output inside the per-channel range of its head's value rows (O is a convex
     combination of V rows)."""
-    c = si.CONFIGS[4]
+    c = si.VIT_L14_336PX_B256
     bits = c.qkv(0)
     qkv = device_qkv(bits)
     import vit_self_attention_b200 as vab
@@ -162,7 +161,7 @@ def test_large_config_sampled_rows_and_hull():
 def test_graph_capture_replay():
     """The call can be captured in a CUDA graph and replayed (pointers stay fixed)."""
     import vit_self_attention_b200 as vab
-    c = si.CONFIGS[2]
+    c = si.VIT_L14_224PX_3VIEWS
     bits = c.qkv(0)
     qkv = device_qkv(bits)
     out = torch.empty((c.B, c.N, c.H, c.d), dtype=torch.bfloat16, device="cuda")
@@ -189,7 +188,7 @@ def test_graph_capture_replay():
 def test_host_buffer_entry():
     """vla_attn_fwd_host: pinned host input -> device -> kernel -> pinned host output."""
     import vit_self_attention_b200 as vab
-    c = si.CONFIGS[3]
+    c = si.SIGLIP_SO400M14_224PX_2VIEWS
     bits = c.qkv(5)
     host_in = torch.from_numpy(bits.view(np.int16).copy()).pin_memory()
     host_out = torch.empty((c.B, c.N, c.H, c.d), dtype=torch.int16).pin_memory()
@@ -230,7 +229,7 @@ def test_host_buffer_entry_pipelined_chunks():
 def test_device_status_clean_and_launch_count():
     import vit_self_attention_b200 as vab
     n0 = vab.vla_attn_launch_count()
-    run_cuda(si.CONFIGS[0].qkv(0), si.CONFIGS[0].scale)
+    run_cuda(si.VIT_B16_112PX_1VIEW.qkv(0), si.VIT_B16_112PX_1VIEW.scale)
     assert vab.vla_attn_launch_count() == n0 + 1
     st, site = vab.vla_attn_last_device_status()
     assert st == 0 and site == 0

@@ -38,23 +38,23 @@ def test_bf16_rounding_matches_torch():
 
 
 def test_moments_and_slot_sigmas():
-    c = si.CONFIGS[3]  # Q, K with variance 2; V with variance 1
+    c = si.SIGLIP_SO400M14_224PX_2VIEWS  # Q, K with variance 2; V with variance 1
     x = si.bf16_bits_to_f32(c.qkv(0)).astype(np.float64)
     q, k, v = x[:, :, 0], x[:, :, 1], x[:, :, 2]
     for arr, var in [(q, 2.0), (k, 2.0), (v, 1.0)]:
         assert abs(arr.mean()) < 0.02
         assert abs(arr.var() - var) < 0.03 * var
-    y = si.bf16_bits_to_f32(si.CONFIGS[1].qkv(0)).astype(np.float64)
+    y = si.bf16_bits_to_f32(si.VIT_B16_224PX_3VIEWS.qkv(0)).astype(np.float64)
     assert abs(y.var() - 1.0) < 0.02
 
 
 def test_config_table():
-    shapes = [(c.B, c.N, c.H, c.d) for c in si.CONFIGS]
+    shapes = [(c.B, c.N, c.H, c.d) for c in si.WORKLOADS]
     assert shapes == [(1, 50, 12, 64), (3, 197, 12, 64), (3, 257, 16, 64), (2, 256, 16, 72),
                       (256, 577, 16, 64)]
-    assert si.CONFIGS[0].scale == 0.125 and si.CONFIGS[0].seed(0) == 0
-    assert [c.calls for c in si.CONFIGS] == [1, 12, 24, 27, 1]
-    assert abs(si.CONFIGS[3].scale - 72 ** -0.5) < 1e-15
-    assert si.CONFIGS[4].flops() == 4 * 256 * 16 * 577 * 577 * 64
-    seeds = {c.seed(i) for c in si.CONFIGS for i in range(c.calls)}
-    assert len(seeds) == sum(c.calls for c in si.CONFIGS)
+    assert si.VIT_B16_112PX_1VIEW.scale == 0.125 and si.VIT_B16_112PX_1VIEW.seed(0) == 0
+    assert [c.calls for c in si.WORKLOADS] == [1, 12, 24, 27, 1]
+    assert abs(si.SIGLIP_SO400M14_224PX_2VIEWS.scale - 72 ** -0.5) < 1e-15
+    assert si.VIT_L14_336PX_B256.flops() == 4 * 256 * 16 * 577 * 577 * 64
+    seeds = {c.seed(i) for c in si.WORKLOADS for i in range(c.calls)}
+    assert len(seeds) == sum(c.calls for c in si.WORKLOADS)
