@@ -22,7 +22,7 @@ def test_encoder_workloads_every_call(c):
         bits = c.qkv(call)
         want = oracle.attention_packed_bf16(bits, c.scale)
         got = run_cuda(bits, c.scale)
-        assert_parity(got, want, f"config {cfg} ({c.name}) call {call}")
+        assert_parity(got, want, f"{c.name} call {call}")
 
 
 # Boundaries of 128-row query tiles / 128-key blocks (d=64) and 112-key blocks (d=72).
