@@ -71,9 +71,12 @@ typedef enum {
  *   B        images (camera views x batch), >= 1.
  *   N        tokens per image (patches + CLS), 1 <= N <= vla_attn_max_tokens(d)
  *            (16384).  Up to 768 tokens for d=64 (560 for d=72) a head's K and
- *            V stay in shared memory for all its query tiles; longer sequences
- *            stream K/V blocks through the shared-memory ring per pair of
- *            query tiles (same result, more L2 traffic).
+ *            V can stay in shared memory for all its query tiles; longer
+ *            sequences, and batches of at least one head per SM whose heads
+ *            have an odd number of 128-row query tiles (their tiles are then
+ *            paired across heads), stream K/V blocks through the
+ *            shared-memory ring per pair of query tiles (same result, more
+ *            L2 traffic).
  *   H        heads, >= 1.
  *   d        head dimension, 64 (ViT-B/16, ViT-L/14) or 72 (SigLIP-So400m/14).
  *   scale    logit scale, usually 1/sqrt(d); finite and > 0.
