@@ -39,9 +39,10 @@ import seeded_inputs as si  # noqa: E402
 WORKLOAD = si.VIT_L14_336PX_B256
 METRIC = "attention TFLOP/s (4*B*H*N^2*d per call) on B200"
 UNIT = "TFLOP/s"
+# Device code of the attention kernel: an ncu summary describes the current kernel
+# only while these files are unchanged (host-side edits do not invalidate it).
 KERNEL_SOURCES = ["vit_self_attention_b200/csrc/attn_kernel.cuh",
-                  "vit_self_attention_b200/csrc/ptx.cuh",
-                  "vit_self_attention_b200/csrc/vla_attn.cu"]
+                  "vit_self_attention_b200/csrc/ptx.cuh"]
 
 
 def kernel_source_hash() -> str:
@@ -64,19 +65,36 @@ def measured_peaks() -> dict:
             "source": "fallback"}
 
 
-def ncu_traffic(workload: str) -> tuple[float | None, str | None]:
-    """DRAM bytes per launch from the committed ncu summary of this kernel and workload,
-    if it was taken on the current kernel source (else None)."""
+def ncu_summary(workload: str) -> tuple[dict, str | None]:
+    """Figures of the committed ncu summary of this kernel and workload, if it was taken
+    on the current kernel sources: ``dram_bytes_per_full_launch`` (DRAM bytes read +
+    written by one launch) and ``tensor_pipe_active_pct`` (sm__pipe_tensor_cycles_active,
+    percent of peak); ({}, None) when there is none."""
     cur = kernel_source_hash()
+    found: dict = {}
+    src = None
     for path in sorted(glob.glob(os.path.join(ROOT, "profiles", "*.md"))):
         with open(path) as f:
             txt = f.read()
         m_w = re.search(r"^workload:\s*(\S+)", txt, re.M)
         m_h = re.search(r"^kernel_source_sha256_16:\s*([0-9a-f]+)", txt, re.M)
-        m_t = re.search(r"^dram_bytes_per_full_launch:\s*([0-9.eE+]+)", txt, re.M)
-        if m_w and m_h and m_t and m_w.group(1) == workload and m_h.group(1) == cur:
-            return float(m_t.group(1)), os.path.relpath(path, ROOT)
-    return None, None
+        if not (m_w and m_h and m_w.group(1) == workload and m_h.group(1) == cur):
+            continue
+        for key in ("dram_bytes_per_full_launch", "tensor_pipe_active_pct"):
+            m = re.search(rf"^{key}:\s*([0-9.eE+]+)", txt, re.M)
+            if m and key not in found:
+                found[key] = float(m.group(1))
+                src = os.path.relpath(path, ROOT) if src is None else src
+    return found, src
+
+
+def ncu_traffic(workload: str) -> tuple[float | None, str | None]:
+    """DRAM bytes per launch from the committed ncu summary of this kernel and workload,
+    if it was taken on the current kernel sources (else None)."""
+    found, src = ncu_summary(workload)
+    if "dram_bytes_per_full_launch" not in found:
+        return None, None
+    return found["dram_bytes_per_full_launch"], src
 
 
 _REASON_BITS = {
@@ -89,7 +107,7 @@ _REASON_BITS = {
 class ClockSampler:
     """Samples SM clock and throttle reasons through NVML while the timed region runs."""
 
-    def __init__(self, device_index: int, period_s: float = 0.005):
+    def __init__(self, device_index: int, period_s: float = 0.001):
         self.samples: list[tuple[int, int]] = []
         self.max_mhz = None
         self._stop = threading.Event()
@@ -299,23 +317,32 @@ def run_ours(args, rank: int, world: int, local_rank: int) -> None:
         e2e_ms = e0.elapsed_time(e1)
 
     ms, e2e_ms = max_over_ranks([ms, e2e_ms], world, dev)
-
-    flops_call = float(c.flops())
-    ms_step = ms / args.steps
-    value = flops_call * world * args.steps / (ms / 1e3) / 1e12
-    e2e_value = flops_call * world * e2e_steps / (e2e_ms / 1e3) / 1e12
-    peaks = measured_peaks()
-    achieved = flops_call / (ms_step / 1e3) / 1e12
-    traffic, traffic_src = ncu_traffic(c.name)
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cb = cpu_oracle_rate(args.cpu_seconds)
         cpu = {k: cb[k] for k in ("value", "unit", "cores", "kind", "sample")}
     if rank != 0:
         return
+    line = build_line(c, world, args.steps, max(3, args.warmup), ms,
+                      None if args.no_e2e else (e2e_ms, e2e_steps, int(bits.nbytes)),
+                      int(launches), clocks.summary(), cpu)
+    print(json.dumps(line), flush=True)
+
+
+def build_line(c, world: int, steps: int, warmup: int, ms: float, e2e, launches: int,
+               clocks: dict | None, cpu: dict | None) -> dict:
+    """The bench's JSON line from the max-over-ranks timings: ``ms`` for ``steps`` device
+    steps of one ``c.B``-image batch per rank, ``e2e`` = (ms, steps, input bytes per step)
+    of the host-buffer leg or None."""
+    flops_call = float(c.flops())
+    ms_step = ms / steps
+    value = flops_call * world * steps / (ms / 1e3) / 1e12
+    peaks = measured_peaks()
+    achieved = flops_call / (ms_step / 1e3) / 1e12
+    prof, prof_src = ncu_summary(c.name)
     line = {
-        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
-        "warmup": max(3, args.warmup), "ms_per_step": ms_step, "higher_is_better": True,
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": steps,
+        "warmup": warmup, "ms_per_step": ms_step, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (seeded splitmix64 Box-Muller, bf16)",
         "config": {"workload": c.name, "B": c.B, "N": c.N, "H": c.H, "d": c.d,
@@ -325,22 +352,29 @@ def run_ours(args, rank: int, world: int, local_rank: int) -> None:
         "images_per_s_24_layers": world * c.B / (ms_step / 1e3) / 24.0,
         "roofline": {"bound": "tensor", "achieved": achieved,
                      "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
-                     "frac": achieved / peaks["bf16_tflops"], "traffic": traffic,
+                     "frac": achieved / peaks["bf16_tflops"],
+                     "traffic": prof.get("dram_bytes_per_full_launch"),
                      "peak_source": f"{peaks['source']} bf16 burst (cuBLAS)",
                      "frac_of_sustained": achieved / peaks["bf16_tflops_sustained"],
                      "hbm_gbs_achieved": c.bytes() / (ms_step / 1e3) / 1e9,
-                     "traffic_source": traffic_src},
+                     "hbm_frac": c.bytes() / (ms_step / 1e3) / 1e9 / peaks["hbm_gbs"],
+                     "tensor_pipe_active_pct": prof.get("tensor_pipe_active_pct"),
+                     "ncu_source": prof_src},
         "cpu_baseline": cpu,
-        "e2e": None if args.no_e2e else {
-            "value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": int(bits.nbytes),
-            "d2h_bytes_per_step": int(c.B * c.N * c.H * c.d * 2),
-            "steps": e2e_steps, "ms_per_step": e2e_ms / e2e_steps,
-            "api": "vla_attn_fwd_host (pinned host buffers)"},
+        "e2e": None,
         "gpu_launches": int(launches),
-        "clocks": clocks.summary(),
+        "clocks": clocks,
         "kernel_source_sha256_16": kernel_source_hash(),
     }
-    print(json.dumps(line), flush=True)
+    if e2e is not None:
+        e2e_ms, e2e_steps, in_bytes = e2e
+        line["e2e"] = {
+            "value": flops_call * world * e2e_steps / (e2e_ms / 1e3) / 1e12, "unit": UNIT,
+            "h2d_bytes_per_step": int(in_bytes),
+            "d2h_bytes_per_step": int(c.B * c.N * c.H * c.d * 2),
+            "steps": e2e_steps, "ms_per_step": e2e_ms / e2e_steps,
+            "api": "vla_attn_fwd_host (pinned host buffers)"}
+    return line
 
 
 def _percentile(xs, q):
@@ -657,6 +691,15 @@ def main() -> None:
         run_block(args)
         return
 
+    if "WORLD_SIZE" not in os.environ and args.gpus > 1:
+        if args.impl == "reference":
+            # The CPU oracle runs on rank 0 alone; the other ranks would do no work.
+            run_reference(args, 0, args.gpus)
+            return
+        # No outer torchrun: start one process per GPU here (same per-rank batch, NCCL
+        # process group over 127.0.0.1), so that --gpus N alone measures N GPUs.
+        launch_ranks(args.gpus, _rank_main, args, backend="nccl")
+        return
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
@@ -668,19 +711,59 @@ def main() -> None:
         return
 
     if world > 1:
-        import datetime
-
-        import torch
-        import torch.distributed as dist
-        torch.cuda.set_device(local_rank)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=torch.device("cuda", local_rank))
+        init_group("nccl", rank, world, local_rank)
     try:
         run_ours(args, rank, world, local_rank)
     finally:
         if world > 1:
             import torch.distributed as dist
             dist.destroy_process_group()
+
+
+def init_group(backend: str, rank: int, world: int, local_rank: int) -> None:
+    """Join the job's process group (MASTER_ADDR / MASTER_PORT from the environment) with
+    a short timeout, so that ranks waiting on a lost peer end with an error."""
+    import datetime
+
+    import torch
+    import torch.distributed as dist
+    timeout = datetime.timedelta(seconds=120)
+    if backend == "nccl":
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", rank=rank, world_size=world, timeout=timeout,
+                                device_id=torch.device("cuda", local_rank))
+    else:
+        dist.init_process_group(backend, rank=rank, world_size=world, timeout=timeout)
+
+
+def _free_port() -> int:
+    import socket
+    with socket.socket() as sk:
+        sk.bind(("127.0.0.1", 0))
+        return sk.getsockname()[1]
+
+
+def _rank_entry(rank: int, world: int, port: int, backend: str, target, target_args) -> None:
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank),
+                      WORLD_SIZE=str(world), LOCAL_RANK=str(rank))
+    import torch.distributed as dist
+    init_group(backend, rank, world, rank)
+    try:
+        target(rank, world, *target_args)
+    finally:
+        dist.destroy_process_group()
+
+
+def launch_ranks(nprocs: int, target, *target_args, backend: str = "nccl") -> None:
+    """Run ``target(rank, world, *target_args)`` in ``nprocs`` spawned processes that form
+    one process group (rank r on GPU r for NCCL); raises if any rank fails."""
+    import torch.multiprocessing as mp
+    mp.spawn(_rank_entry, args=(nprocs, _free_port(), backend, target, target_args),
+             nprocs=nprocs, join=True)
+
+
+def _rank_main(rank: int, world: int, args) -> None:
+    run_ours(args, rank, world, rank)
 
 
 if __name__ == "__main__":

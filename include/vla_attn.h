@@ -99,13 +99,23 @@ int vla_attn_fwd(const void* q, const void* k, const void* v, void* o,
  * vla_attn_fwd on the whole batch, and the host result is valid once
  * `stream` has been synchronised.  Host buffers should be pinned
  * (cudaHostAlloc / cudaHostRegister) for the copies to be asynchronous.
- * Same argument rules and status codes as vla_attn_fwd.  Allocates no memory;
+ * Same argument rules and status codes as vla_attn_fwd; the device buffers are
+ * range-checked (qkv_dev must hold 3*B*N*H*d and o_dev B*N*H*d bf16 elements
+ * inside one device allocation each, and they must not overlap) before the
+ * first copy is enqueued, so an argument error leaves nothing enqueued.
+ * Allocates no memory;
  * the first pipelined call on a device creates the copy-out stream and two
  * events, which live as long as the process.  Calls are serialised on a
  * library lock while they enqueue.
  */
 int vla_attn_fwd_host(const void* qkv_host, void* o_host, void* qkv_dev, void* o_dev,
                       int B, int N, int H, int d, float scale, void* stream);
+
+/*
+ * Utility calls.  The pages describe the operation only; the status calls
+ * below, the launch counter and the testing hooks are this library's own
+ * plumbing and follow no passage of them.
+ */
 
 /* Human-readable text for a status code (static storage, never NULL). */
 const char* vla_attn_strerror(int status);
@@ -114,7 +124,13 @@ const char* vla_attn_strerror(int status);
  * Synchronises `stream` and returns the device-side status of the kernels run
  * since the last reset: VLA_ATTN_OK, or VLA_ATTN_ERR_TIMEOUT if a bounded wait
  * ran out (the output of that launch is then undefined).  `site`, if non-NULL,
- * receives the code of the first wait that ran out (0 if none).
+ * receives the code of the first wait that ran out (0 if none): 1-3 the TMA
+ * producer (Q slot, K block, V block), 11-15 the tensor-core issuers (Q, K,
+ * V, P, S read out), 21-22 the softmax warps (S, P V progress), 31 a drain
+ * wait, 41 the testing stall.  This extends the plain status call
+ * vla_attn_last_device_status(stream) by the optional `site` out-parameter
+ * (pass NULL for the plain form).  The status word is always kept; reading
+ * it costs a stream synchronisation, so call it outside timed regions.
  */
 int vla_attn_last_device_status(void* stream, int* site);
 

@@ -44,6 +44,36 @@ def test_max_over_ranks_and_seeds_gloo():
     assert res[10] != res[11]  # each rank draws a different batch
 
 
+def _stub_rank(rank, world, out):
+    """One rank of a two-rank job with a stubbed step: rank r 'took' 10 + 5 r ms for 4
+    steps; the line comes from the max over ranks, as bench.py's own ranks build it."""
+    sys.path.insert(0, ROOT)
+    import bench
+    ms, e2e_ms = bench.max_over_ranks([10.0 + 5.0 * rank, 40.0 - rank], world, "cpu")
+    if rank == 0:
+        out["line"] = bench.build_line(bench.WORKLOAD, world, 4, 3, ms, (e2e_ms, 2, 123), 4,
+                                       None, None)
+    out[f"env{rank}"] = (os.environ["RANK"], os.environ["WORLD_SIZE"], os.environ["MASTER_ADDR"])
+
+
+def test_spawned_ranks_report_one_line_over_both_ranks():
+    """bench.launch_ranks (used by --gpus N without an outer torchrun) forms a two-rank
+    gloo group; the reported value counts both ranks' images over the slower rank's time."""
+    sys.path.insert(0, ROOT)
+    import bench
+    with mp.Manager() as m:
+        out = m.dict()
+        bench.launch_ranks(2, _stub_rank, out, backend="gloo")
+        res = dict(out)
+    line = res["line"]
+    c = bench.WORKLOAD
+    assert line["n_gpus"] == 2 and line["steps"] == 4 and line["scaling"] == "weak"
+    assert abs(line["ms_per_step"] - 15.0 / 4) < 1e-12  # the slower rank
+    assert abs(line["value"] - c.flops() * 2 * 4 / 15e-3 / 1e12) < 1e-9 * line["value"]
+    assert abs(line["e2e"]["ms_per_step"] - 40.0 / 2) < 1e-12
+    assert res["env0"] == ("0", "2", "127.0.0.1") and res["env1"] == ("1", "2", "127.0.0.1")
+
+
 def test_max_over_ranks_single_rank_is_identity():
     sys.path.insert(0, ROOT)
     import bench

@@ -46,3 +46,25 @@ def test_static_workspace_linear_matches_regular_entry_point():
         torch.cuda.synchronize()
         assert torch.isfinite(y_static.float()).all()
         assert torch.equal(y_static, y_regular), f"M={M} K={K} N={N}"
+
+
+def test_static_workspace_linear_warm_calls_allocate_nothing():
+    """After one warm call (which does the per-device set-up), further calls change
+    neither torch's allocated bytes nor the device's free memory."""
+    import vit_self_attention_b200 as vab
+    from cuda.bindings import runtime as cudart
+    M, K, N = 771, 1024, 3072
+    x, w, b, r = _case(M, K, N, 3000, True)
+    y = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+    assert vab.vla_linear_fwd_static(x, w, b, r, y, M, K, N) == vab.OK
+    torch.cuda.synchronize()
+    alloc0 = torch.cuda.memory_allocated()
+    err, free0, _ = cudart.cudaMemGetInfo()
+    assert int(err) == 0
+    for _ in range(5):
+        assert vab.vla_linear_fwd_static(x, w, b, r, y, M, K, N) == vab.OK
+    torch.cuda.synchronize()
+    err, free1, _ = cudart.cudaMemGetInfo()
+    assert int(err) == 0
+    assert torch.cuda.memory_allocated() == alloc0
+    assert free1 == free0, f"device free memory changed by {free0 - free1} bytes"

@@ -265,17 +265,26 @@ __device__ __align__(256) unsigned char g_static_workspace[kStaticWorkspaceBytes
 
 std::mutex g_static_ws_mutex;
 void* g_static_ws_addr[kMaxDevices] = {};
+CUcontext g_static_ws_ctx[kMaxDevices] = {};
 
-// Device address of this device's static workspace (looked up once per device).
+// Device address of this device's static workspace.  A module global's address belongs
+// to the context the module is loaded in, so the address is cached together with the
+// context that was current when it was looked up, and looked up again whenever another
+// context is current (a non-primary context, or the primary one after a device reset).
 int static_workspace(int dev, void** out) {
+  const DriverFns& fns = driver_fns();
+  if (fns.ctx_current == nullptr) return VLA_ATTN_ERR_CUDA;
+  CUcontext ctx = nullptr;
+  if (fns.ctx_current(&ctx) != CUDA_SUCCESS || ctx == nullptr) return VLA_ATTN_ERR_CUDA;
   std::lock_guard<std::mutex> lock(g_static_ws_mutex);
-  if (g_static_ws_addr[dev] == nullptr) {
+  if (g_static_ws_addr[dev] == nullptr || g_static_ws_ctx[dev] != ctx) {
     void* p = nullptr;
     if (cudaGetSymbolAddress(&p, g_static_workspace) != cudaSuccess || p == nullptr) {
       (void)cudaGetLastError();
       return VLA_ATTN_ERR_CUDA;
     }
     g_static_ws_addr[dev] = p;
+    g_static_ws_ctx[dev] = ctx;
   }
   *out = g_static_ws_addr[dev];
   return VLA_ATTN_OK;

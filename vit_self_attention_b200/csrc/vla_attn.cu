@@ -32,6 +32,7 @@ std::atomic<int> g_test_stall{0};
 struct DriverFns {
   PFN_cuTensorMapEncodeTiled_v12000 encode = nullptr;
   PFN_cuPointerGetAttribute_v4000 ptr_attr = nullptr;
+  PFN_cuCtxGetCurrent_v4000 ctx_current = nullptr;
 };
 
 const DriverFns& driver_fns() {
@@ -49,6 +50,10 @@ const DriverFns& driver_fns() {
             cudaSuccess &&
         q == cudaDriverEntryPointSuccess)
       fns.ptr_attr = reinterpret_cast<PFN_cuPointerGetAttribute_v4000>(fn);
+    fn = nullptr;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &fn, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fns.ctx_current = reinterpret_cast<PFN_cuCtxGetCurrent_v4000>(fn);
   });
   return fns;
 }
@@ -322,6 +327,18 @@ int vla_attn_fwd_host(const void* qkv_host, void* o_host, void* qkv_dev, void* o
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const size_t img_out = static_cast<size_t>(N) * H * d * 2u;  // bytes of one image's O
   const size_t img_in = 3u * img_out;                           // and of its packed QKV
+  // The device buffers must hold the whole batch and must not overlap, checked before
+  // the first copy is enqueued (as vla_attn_fwd checks its buffers before its launch).
+  {
+    const DriverFns& fns = driver_fns();
+    if (fns.encode == nullptr || fns.ptr_attr == nullptr) return VLA_ATTN_ERR_CUDA;
+    uintptr_t in_lo = 0, in_hi = 0, out_lo = 0, out_hi = 0;
+    if ((rc = check_device_range(fns, qkv_dev, img_in * B, dev, &in_lo, &in_hi)) != VLA_ATTN_OK)
+      return rc;
+    if ((rc = check_device_range(fns, o_dev, img_out * B, dev, &out_lo, &out_hi)) != VLA_ATTN_OK)
+      return rc;
+    if (out_lo < in_hi && in_lo < out_hi) return VLA_ATTN_ERR_MEMORY;
+  }
   // Chunks of whole images, each with at least 4 heads per SM so that every
   // launch still fills the GPU; a batch smaller than two chunks goes in one.
   const long long min_heads = 4ll * di.sm_count;
