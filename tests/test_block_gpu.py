@@ -5,14 +5,15 @@ Stage-wise: every GPU stage is compared with the oracle on identical bf16 inputs
 (the GPU's own bf16 output of the previous stage feeds the oracle's next stage).
 Tolerance: the attention stage keeps the attention bound (max |err| <= 2e-2,
 mean |err| <= 2e-3); LayerNorm and linear outputs use the bound derived from their
-arithmetic (bf16 rounding of an fp32 result, possibly twice -- GEMM + bias, then the
-residual sum -- each at most 2^-9 of what it rounds: elementwise
-|err| <= 2^-7 (|x w^T + b| + |res|) + 2^-9, mean error <= 2^-8 of the mean magnitude),
-since their outputs reach |y| ~ 6 where one bf16 ulp is 0.03.  The residual stream of
-the fused add + LayerNorm is compared bit for bit (one rounding of an exact sum).  The
-GELU output adds the error of the epilogue's tanh, taken as at most 2^-10 absolute
-(a hardware tanh approximation's bound), i.e. 2^-10 |a| / 2 for pre-activation a, which
-the magnitude |y| + |a| / 8 covers.
+arithmetic: the output is an fp32 result (the GEMM's accumulation with bias, GELU and
+residual applied in the same fp32 epilogue) rounded to bf16 once, at most 2^-9 of what it
+rounds, so elementwise |err| <= 2^-8 (|x w^T + b| + |res|) + 2^-10 and the mean error
+<= 2^-9 of the mean magnitude (an absolute bound like the attention's would not fit:
+these outputs reach |y| ~ 6, where one bf16 ulp is 0.03).  The residual stream of the
+fused add + LayerNorm is compared bit for bit (one rounding of an exact sum).  The GELU
+output adds the error of the epilogue's tanh, the hardware approximation's absolute
+error below 2^-10.9, i.e. under 2^-11 |a| for pre-activation a, which the magnitude
+|y| + |a| / 8 covers.
 """
 import math
 
@@ -99,6 +100,48 @@ def test_linear_bias_residual_variants(M, K, N, bias, res):
     want = oracle.linear_bf16(x, w, b if bias else None, r)
     assert_close_bf16(f64(got), want, f"linear M={M} K={K} N={N} bias={bias} res={res}",
                       mag=residual_magnitude(x, w, b if bias else None, r))
+
+
+@pytest.mark.parametrize("M,K,N,res,ws", [
+    (591, 3072, 768, True, True),     # ViT-B/16 fc2 (3 views): few tiles, split K
+    (591, 3072, 768, True, False),    # the same without a workspace: one part per tile
+    (512, 4304, 1152, True, True),    # SigLIP fc2: K not a multiple of 64, split K
+    (4096, 1024, 3072, False, True),  # 256-wide tiles, several waves over the SMs
+    (300, 136, 72, True, True),       # K and N ending inside one 64-wide step / tile
+    (2000, 768, 2304, False, True),   # 128-wide tiles
+])
+def test_linear_tile_widths_and_split_k(M, K, N, res, ws):
+    """The GEMM's tile-width choices (256 / 128 / 64 columns) and its split-K path (fp32
+    partial sums in the caller's workspace, added up in split order by the last arrival)
+    against the oracle; without a workspace the same shape runs unsplit."""
+    import vit_self_attention_b200 as vab
+    x, w, b = linear_inputs(M, K, N, 900 + M + K + N)
+    r = si.normal_bf16(950 + M, (M, N)) if res else None
+    y = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+    wsb = vab.vla_linear_workspace_bytes() if ws else 0
+    wst = torch.empty(max(wsb, 1), dtype=torch.uint8, device="cuda") if ws else None
+    vab.vla_linear_fwd(dev(x), dev(w), dev(b), dev(r) if res else None, y, M, K, N, wst, wsb)
+    torch.cuda.synchronize()
+    assert_close_bf16(f64(y), oracle.linear_bf16(x, w, b, r),
+                      f"linear M={M} K={K} N={N} res={res} workspace={ws}",
+                      mag=residual_magnitude(x, w, b, r))
+
+
+def test_linear_gelu_split_k():
+    """fc1 + GELU on a shape with few tiles (split K) and on the same shape unsplit: both
+    against the oracle, and the two GPU results equal (same sums, different order only
+    within fp32)."""
+    import vit_self_attention_b200 as vab
+    M, K, N = 200, 2048, 256
+    x, w, b = linear_inputs(M, K, N, 1200)
+    want = oracle.linear_gelu_bf16(x, w, b)
+    a = np.abs(oracle.linear_bf16(x, w, b))
+    for wsb in (vab.vla_linear_workspace_bytes(), 0):
+        wst = torch.empty(max(wsb, 1), dtype=torch.uint8, device="cuda")
+        y = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+        vab.vla_linear_gelu_fwd(dev(x), dev(w), dev(b), y, M, K, N, wst if wsb else None, wsb)
+        torch.cuda.synchronize()
+        assert_close_bf16(f64(y), want, f"fc1 + GELU workspace={wsb}", mag=np.abs(want) + a / 8)
 
 
 def test_linear_in_place_residual():
@@ -371,3 +414,105 @@ def test_encoder_layers_graph_capture():
     g.replay()
     torch.cuda.synchronize()
     assert torch.equal(xg, eager)
+
+
+def _layer_weights(W, F, seed):
+    n = lambda s, shape, m, sd: si.normal_bf16(seed + s, shape, m, sd)
+    return {"g": n(0, (W,), 1.0, 0.1), "be": n(1, (W,), 0.0, 0.1),
+            "wq": n(2, (3 * W, W), 0.0, 1.0 / math.sqrt(W)), "bq": n(3, (3 * W,), 0.0, 0.1),
+            "wo": n(4, (W, W), 0.0, 1.0 / math.sqrt(W)), "bo": n(5, (W,), 0.0, 0.1),
+            "g2": n(6, (W,), 1.0, 0.1), "be2": n(7, (W,), 0.0, 0.1),
+            "w1": n(8, (F, W), 0.0, 1.0 / math.sqrt(W)), "b1": n(9, (F,), 0.0, 0.1),
+            "w2": n(10, (W, F), 0.0, 1.0 / math.sqrt(F)), "b2": n(11, (W,), 0.0, 0.1)}
+
+
+def _oracle_layer(x, p, c):
+    """One pre-norm encoder layer in the oracle, every stage's fp64 result rounded to bf16
+    before the next stage reads it (the precision at which the layers hand over)."""
+    W = c.H * c.d
+    r = oracle.round_bf16
+    xn = r(oracle.layernorm_bf16(x, p["g"], p["be"], 1e-6))
+    qkv = r(oracle.linear_bf16(xn, p["wq"], p["bq"]))
+    o = r(oracle.attention_packed_bf16(qkv.reshape(c.B, c.N, 3, c.H, c.d), c.scale))
+    h = r(oracle.linear_bf16(o.reshape(c.B * c.N, W), p["wo"], p["bo"], x))
+    hn = r(oracle.layernorm_bf16(h, p["g2"], p["be2"], 1e-6))
+    a = r(oracle.linear_gelu_bf16(hn, p["w1"], p["b1"]))
+    return r(oracle.linear_bf16(a, p["w2"], p["b2"], h))
+
+
+def test_encoder_chain_against_oracle_chain_eager_and_graph():
+    """Four whole encoder layers of the ViT-B/16 224 px workload (3 views: 591 tokens,
+    width 768, MLP 3072, seeded weights per layer), run eagerly and replayed from one CUDA
+    graph, against the oracle chain fed the same bf16 weights (each oracle stage reading the
+    previous oracle stage's bf16-rounded output).
+
+    Bound for L layers: each layer rounds the residual stream twice, and two correct
+    evaluations whose pre-rounding values differ within the stage bounds can round an
+    element to neighbouring bf16 values, one spacing (at most 2^-7 of its magnitude) apart;
+    the residual path carries such a difference forward, and the branches add their own
+    stage errors on top.  So the difference grows about linearly with L: mean |err| <=
+    2^-8 L mean|x_L| and max |err| <= 2^-4 L rms(x_L) for the final stream x_L (a float32
+    chain rounded at the same points differs from the oracle chain by 0.0013 L mean|x_L| in
+    mean and 0.025-0.05 rms(x_L) at most for L <= 4)."""
+    import vit_self_attention_b200 as vab
+    c = si.VIT_B16_224PX_3VIEWS
+    L, W, F = 4, c.H * c.d, 3072
+    M = c.B * c.N
+    params = [_layer_weights(W, F, 2000 + 13 * i) for i in range(L)]
+    x0 = si.normal_bf16(1999, (M, W))
+    want = x0
+    for p in params:
+        want = _oracle_layer(want, p, c)
+    want64 = si.bf16_bits_to_f32(want).astype(np.float64)
+
+    dp = [{k: dev(v) for k, v in p.items()} for p in params]
+    ws = torch.empty(vab.vla_linear_workspace_bytes(), dtype=torch.uint8, device="cuda")
+    xs = [dev(x0)] + [torch.empty((M, W), dtype=torch.bfloat16, device="cuda")
+                      for _ in range(2 * L)]
+    xn = torch.empty((M, W), dtype=torch.bfloat16, device="cuda")
+    qkv = torch.empty((M, 3 * W), dtype=torch.bfloat16, device="cuda")
+    o = torch.empty((c.B, c.N, c.H, c.d), dtype=torch.bfloat16, device="cuda")
+    a = torch.empty((M, F), dtype=torch.bfloat16, device="cuda")
+
+    def encoder(stream=None):
+        for i, q in enumerate(dp):
+            h_in, h_mid, h_out = xs[2 * i], xs[2 * i + 1], xs[2 * i + 2]
+            vab.layernorm(h_in, q["g"], q["be"], 1e-6, out=xn, stream=stream)
+            vab.linear(xn, q["wq"], q["bq"], out=qkv, workspace=ws, stream=stream)
+            vab.attention(qkv.view(c.B, c.N, 3, c.H, c.d), c.scale, out=o, stream=stream)
+            vab.linear(o.view(M, W), q["wo"], q["bo"], h_in, out=h_mid, workspace=ws,
+                       stream=stream)
+            vab.layernorm(h_mid, q["g2"], q["be2"], 1e-6, out=xn, stream=stream)
+            vab.linear_gelu(xn, q["w1"], q["b1"], out=a, workspace=ws, stream=stream)
+            vab.linear(a, q["w2"], q["b2"], h_mid, out=h_out, workspace=ws, stream=stream)
+
+    def check(got, what):
+        got = f64(got)
+        assert np.all(np.isfinite(got)), what
+        err = np.abs(got - want64)
+        rms = float(np.sqrt((want64 ** 2).mean()))
+        mean_bound = 2.0 ** -8 * L * float(np.abs(want64).mean())
+        assert float(err.mean()) <= mean_bound, f"{what}: mean|err| {err.mean():.3e} > {mean_bound:.3e}"
+        assert float(err.max()) <= 2.0 ** -4 * L * rms, f"{what}: max|err| {err.max():.3e}"
+
+    encoder()
+    torch.cuda.synchronize()
+    eager = xs[-1].clone()
+    check(eager, "eager encoder chain")
+
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        encoder(s)  # warm-up on the capture stream
+    torch.cuda.current_stream().wait_stream(s)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s):
+        encoder(s)
+    for t in xs[1:]:
+        t.zero_()
+    g.replay()
+    torch.cuda.synchronize()
+    check(xs[-1], "graph-replayed encoder chain")
+    assert torch.equal(xs[-1], eager), "graph replay differs from the eager run"
+    del g

@@ -12,11 +12,9 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libvla_attn.so")
 SOURCES = [os.path.join(CSRC, "vla_attn.cu")]
-DEPS = SOURCES + [os.path.join(CSRC, f) for f in ("attn_kernel.cuh", "ptx.cuh", "block_ops.cuh")] + [
+DEPS = SOURCES + [os.path.join(CSRC, f) for f in ("attn_kernel.cuh", "ptx.cuh", "block_ops.cuh",
+                                                  "gemm_kernel.cuh")] + [
     os.path.join(INCLUDE, "vla_attn.h")]
-
-
-CUDA_LIB = "/usr/local/cuda/lib64"  # libcublasLt (the linear layers' GEMM)
 
 
 def nvcc() -> str:
@@ -29,7 +27,7 @@ def nvcc() -> str:
 def flags(verbose_ptxas: bool = False):
     f = ["-gencode", "arch=compute_100a,code=sm_100a", "-lineinfo", "-O3", "-std=c++17",
          "--expt-relaxed-constexpr", "-Xcompiler", "-fPIC", "-shared", "-I", INCLUDE, "-I", CSRC,
-         "-lcublasLt", "-Xlinker", "-rpath", "-Xlinker", CUDA_LIB]
+         ]
     if verbose_ptxas:
         f += ["-Xptxas", "-v"]
     return f

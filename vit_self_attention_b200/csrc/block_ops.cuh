@@ -16,25 +16,22 @@
 //
 //   Linear layer with bias and optional residual, nn.Linear weight layout
 //   [N, K] (the pages' weight(K,N) transposed):
-//     y[m,n] = sum_k x[m,k] * w[n,k] + bias[n] + res[m,n]
-//   (same page, section 3, CUDA custom operators: cublasLt fused GEMM + bias
-//   (+ residual) in one launch; "Pi0 VLA deployment tutorial", section 3.2:
-//   the block's qkv linear feeds the attention.)  A plain GEMM with a bias
-//   epilogue, so it is a cuBLASLt call (tensor cores, bias in the epilogue,
-//   residual as C with beta = 1); the row-major product is computed as the
-//   column-major y^T = w . x^T.  For the qkv linear, N = 3 H d and y is
-//   exactly the packed [B, tokens, 3, H, d] input of the attention kernel.
-//   The MLP's first layer applies GELU (the tanh form) in the same epilogue
-//   (same page, Triton fused kernels: matrix multiply + bias + activation).
+//     y[m,n] = act(sum_k x[m,k] * w[n,k] + bias[n]) + res[m,n]
+//   (same page, section 3, CUDA custom operators: GEMM + bias (+ residual)
+//   in one launch; section 1: matrix multiply + bias + activation; "Pi0 VLA
+//   deployment tutorial", section 3.2: the block's qkv linear feeds the
+//   attention.)  The hand-written tcgen05 GEMM of gemm_kernel.cuh with the
+//   bias, the GELU (tanh form) and the residual add in its epilogue.  For the
+//   qkv linear, N = 3 H d and y is exactly the packed [B, tokens, 3, H, d]
+//   input of the attention kernel.
 //
 // This header is included by vla_attn.cu after its host helpers (device
 // checks, pointer-range checks) and shares them.
 #pragma once
 
-#include <cublasLt.h>
+#include <algorithm>
 
-#include <map>
-#include <tuple>
+#include "gemm_kernel.cuh"
 
 namespace vla {
 
@@ -186,80 +183,143 @@ int dispatch_layernorm(const void* x, const void* r, const void* gamma, const vo
   }
 }
 
-// cuBLASLt state: one handle per process, one plan (descriptors + heuristic
-// algorithm) per shape, device and epilogue.
-struct LtPlan {
-  cublasLtMatmulDesc_t op = nullptr;
-  cublasLtMatrixLayout_t a = nullptr, b = nullptr, c = nullptr;
-  cublasLtMatmulAlgo_t algo{};
+// ---------------------------------------------------------------- linear
+// 2-D tensor map of a row-major [rows, K] bf16 matrix, box {64, box_rows},
+// 128-byte swizzle (the K-major operand layout of the GEMM's MMAs).
+int encode_2d(const DriverFns& fns, CUtensorMap* map, const void* base, int K, int rows,
+              uint32_t box_rows) {
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(rows)};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(K) * 2ull};
+  const cuuint32_t box[2] = {static_cast<cuuint32_t>(vla::gemm::kBK), box_rows};
+  const cuuint32_t elem_strides[2] = {1u, 1u};
+  const CUresult rc = fns.encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base),
+                                 dims, strides, box, elem_strides, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                                 CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                                 CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return rc == CUDA_SUCCESS ? VLA_ATTN_OK : VLA_ATTN_ERR_CUDA;
+}
+
+// How a linear layer is cut into work: tile width BN and K parts.
+struct LinearPlan {
+  int bn = 256;
+  int splits = 1;
+  int tiles_m = 0, tiles_n = 0, ksteps = 0, ksteps_per_split = 0;
+  size_t workspace_needed = 0;  // partial sums + arrival counters (0 without split K)
 };
 
-std::mutex g_lt_mutex;
-cublasLtHandle_t g_lt = nullptr;
-std::map<std::tuple<int, int, int, int, int, int, int, size_t>, LtPlan> g_lt_plans;
+// Tile width: the fewest waves of tiles over the SMs weighted by the tile's
+// MMA time (proportional to BN), wider tiles on ties (more reuse per byte
+// loaded).  Split K when the tiles fill at most half the SMs and the caller's
+// workspace holds the partial sums.
+LinearPlan plan_linear(int M, int K, int N, int sm_count, size_t workspace_bytes) {
+  LinearPlan pl;
+  pl.tiles_m = (M + vla::gemm::kBM - 1) / vla::gemm::kBM;
+  pl.ksteps = (K + vla::gemm::kBK - 1) / vla::gemm::kBK;
+  long long best = -1;
+  for (int bn : {256, 128, 64}) {
+    const long long tiles = static_cast<long long>(pl.tiles_m) * ((N + bn - 1) / bn);
+    const long long cost = ((tiles + sm_count - 1) / sm_count) * bn;
+    if (best < 0 || cost < best) {
+      best = cost;
+      pl.bn = bn;
+    }
+  }
+  pl.tiles_n = (N + pl.bn - 1) / pl.bn;
+  const long long tiles = static_cast<long long>(pl.tiles_m) * pl.tiles_n;
+  pl.ksteps_per_split = pl.ksteps;
+  if (2 * tiles <= sm_count && pl.ksteps >= 8) {
+    int splits = static_cast<int>(sm_count / tiles);
+    splits = std::min(splits, pl.ksteps / 4);
+    splits = std::min(splits, 16);
+    while (splits > 1) {
+      const int per = (pl.ksteps + splits - 1) / splits;
+      const int used = (pl.ksteps + per - 1) / per;  // no empty part
+      const size_t need = static_cast<size_t>(used) * tiles * vla::gemm::kBM * pl.bn * 4u +
+                          static_cast<size_t>(tiles) * 4u * sizeof(unsigned int);
+      if (need <= workspace_bytes) {
+        pl.splits = used;
+        pl.ksteps_per_split = per;
+        pl.workspace_needed = need;
+        break;
+      }
+      --splits;
+    }
+  }
+  return pl;
+}
 
-// Builds (once) the plan of y^T[N, M] = act(w[N, K] . x^T[K, M] (+ bias)) (+ res^T),
-// act = GELU (cuBLASLt's epilogue, the tanh form) or the identity.
-int lt_plan(int dev, int M, int K, int N, bool bias, bool res, bool gelu, size_t ws,
-            LtPlan** out) {
-  if (g_lt == nullptr && cublasLtCreate(&g_lt) != CUBLAS_STATUS_SUCCESS) return VLA_ATTN_ERR_CUDA;
-  const auto key = std::make_tuple(dev, M, K, N, bias ? 1 : 0, res ? 1 : 0, gelu ? 1 : 0, ws);
-  auto it = g_lt_plans.find(key);
-  if (it != g_lt_plans.end()) {
-    *out = &it->second;
-    return VLA_ATTN_OK;
+template <int BN>
+int launch_linear_bn(const DriverFns& fns, const DeviceInfo& di, int dev, const LinearPlan& pl,
+                     const void* x, const void* w, const void* bias, const void* res, void* y,
+                     int M, int K, int N, int act, void* workspace, cudaStream_t stream) {
+  using G = vla::gemm::GemmGeom<BN>;
+  vla::gemm::GemmParams prm;
+  std::memset(&prm, 0, sizeof(prm));
+  int rc = encode_2d(fns, &prm.tm_a, x, K, M, vla::gemm::kBM);
+  if (rc != VLA_ATTN_OK) return rc;
+  rc = encode_2d(fns, &prm.tm_b, w, K, N, static_cast<uint32_t>(BN));
+  if (rc != VLA_ATTN_OK) return rc;
+  int stages = (di.max_smem_optin - static_cast<int>(vla::gemm::kBarrierBytes + 1024u)) /
+               static_cast<int>(G::kStageBytes);
+  if (stages > vla::gemm::kMaxStages) stages = vla::gemm::kMaxStages;
+  if (stages < 2) return VLA_ATTN_ERR_DEVICE;
+  const uint32_t smem = vla::gemm::gemm_smem_bytes<BN>(stages);
+  {
+    static int attr[kMaxDevices] = {};
+    std::lock_guard<std::mutex> lock(g_dev_mutex);
+    if (attr[dev] < static_cast<int>(smem)) {
+      if (cudaFuncSetAttribute(vla::gemm::linear_kernel<BN>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               static_cast<int>(smem)) != cudaSuccess)
+        return VLA_ATTN_ERR_CUDA;
+      attr[dev] = static_cast<int>(smem);
+    }
   }
-  LtPlan pl;
-  bool ok = cublasLtMatmulDescCreate(&pl.op, CUBLAS_COMPUTE_32F, CUDA_R_32F) ==
-            CUBLAS_STATUS_SUCCESS;
-  const cublasOperation_t ta = CUBLAS_OP_T, tb = CUBLAS_OP_N;
-  const cublasLtEpilogue_t epi =
-      gelu ? (bias ? CUBLASLT_EPILOGUE_GELU_BIAS : CUBLASLT_EPILOGUE_GELU)
-           : (bias ? CUBLASLT_EPILOGUE_BIAS : CUBLASLT_EPILOGUE_DEFAULT);
-  const cudaDataType_t bias_type = CUDA_R_16BF;
-  ok = ok && cublasLtMatmulDescSetAttribute(pl.op, CUBLASLT_MATMUL_DESC_TRANSA, &ta,
-                                            sizeof(ta)) == CUBLAS_STATUS_SUCCESS;
-  ok = ok && cublasLtMatmulDescSetAttribute(pl.op, CUBLASLT_MATMUL_DESC_TRANSB, &tb,
-                                            sizeof(tb)) == CUBLAS_STATUS_SUCCESS;
-  ok = ok && cublasLtMatmulDescSetAttribute(pl.op, CUBLASLT_MATMUL_DESC_EPILOGUE, &epi,
-                                            sizeof(epi)) == CUBLAS_STATUS_SUCCESS;
-  if (bias)
-    ok = ok && cublasLtMatmulDescSetAttribute(pl.op, CUBLASLT_MATMUL_DESC_BIAS_DATA_TYPE,
-                                              &bias_type, sizeof(bias_type)) ==
-                   CUBLAS_STATUS_SUCCESS;
-  // w as stored ([N, K] row-major) is a column-major K x N matrix (ld K);
-  // x ([M, K] row-major) a column-major K x M one; y and res column-major N x M.
-  ok = ok && cublasLtMatrixLayoutCreate(&pl.a, CUDA_R_16BF, K, N, K) == CUBLAS_STATUS_SUCCESS;
-  ok = ok && cublasLtMatrixLayoutCreate(&pl.b, CUDA_R_16BF, K, M, K) == CUBLAS_STATUS_SUCCESS;
-  ok = ok && cublasLtMatrixLayoutCreate(&pl.c, CUDA_R_16BF, N, M, N) == CUBLAS_STATUS_SUCCESS;
-  if (ok) {
-    cublasLtMatmulPreference_t pref = nullptr;
-    ok = cublasLtMatmulPreferenceCreate(&pref) == CUBLAS_STATUS_SUCCESS &&
-         cublasLtMatmulPreferenceSetAttribute(pref, CUBLASLT_MATMUL_PREF_MAX_WORKSPACE_BYTES, &ws,
-                                              sizeof(ws)) == CUBLAS_STATUS_SUCCESS;
-    cublasLtMatmulHeuristicResult_t h{};
-    int found = 0;
-    ok = ok && cublasLtMatmulAlgoGetHeuristic(g_lt, pl.op, pl.a, pl.b, pl.c, pl.c, pref, 1, &h,
-                                              &found) == CUBLAS_STATUS_SUCCESS &&
-         found > 0;
-    if (pref != nullptr) cublasLtMatmulPreferenceDestroy(pref);
-    if (ok) pl.algo = h.algo;
+  prm.bias = static_cast<const __nv_bfloat16*>(bias);
+  prm.res = static_cast<const __nv_bfloat16*>(res);
+  prm.y = static_cast<__nv_bfloat16*>(y);
+  prm.M = M;
+  prm.N = N;
+  prm.K = K;
+  prm.tiles_m = pl.tiles_m;
+  prm.tiles_n = pl.tiles_n;
+  prm.splits = pl.splits;
+  prm.ksteps = pl.ksteps;
+  prm.ksteps_per_split = pl.ksteps_per_split;
+  prm.num_work = pl.tiles_m * pl.tiles_n * pl.splits;
+  prm.stages = stages;
+  prm.act = act;
+  const unsigned long long lim = g_wait_limit_ns.load();
+  prm.wait_limit_ns = lim == 0 ? kDefaultWaitLimitNs : lim;
+  if (pl.splits > 1) {
+    // Partial sums first, then the arrival counters, which must start at zero.
+    const size_t tiles = static_cast<size_t>(pl.tiles_m) * pl.tiles_n;
+    const size_t part_bytes =
+        static_cast<size_t>(pl.splits) * tiles * vla::gemm::kBM * BN * 4u;
+    prm.partial = static_cast<float*>(workspace);
+    prm.counters = reinterpret_cast<unsigned int*>(static_cast<char*>(workspace) + part_bytes);
+    if (cudaMemsetAsync(prm.counters, 0, tiles * 4u * sizeof(unsigned int), stream) !=
+        cudaSuccess)
+      return VLA_ATTN_ERR_CUDA;
   }
-  if (!ok) {
-    if (pl.op) cublasLtMatmulDescDestroy(pl.op);
-    if (pl.a) cublasLtMatrixLayoutDestroy(pl.a);
-    if (pl.b) cublasLtMatrixLayoutDestroy(pl.b);
-    if (pl.c) cublasLtMatrixLayoutDestroy(pl.c);
+  const int grid = prm.num_work < di.sm_count ? prm.num_work : di.sm_count;
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(static_cast<unsigned>(grid), 1, 1);
+  cfg.blockDim = dim3(vla::gemm::kThreads, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  if (cudaLaunchKernelEx(&cfg, vla::gemm::linear_kernel<BN>, prm) != cudaSuccess) {
+    (void)cudaGetLastError();
     return VLA_ATTN_ERR_CUDA;
   }
-  auto ins = g_lt_plans.emplace(key, pl);
-  *out = &ins.first->second;
+  g_launches.fetch_add(1);
   return VLA_ATTN_OK;
 }
 
 constexpr size_t kLinearWorkspaceBytes = 32u << 20;
 
-// Fixed cuBLASLt workspace of vla_linear_fwd_static: one per device context.
+// Fixed workspace of vla_linear_fwd_static (split-K partial sums and arrival
+// counters): one per device context.
 constexpr size_t kStaticWorkspaceBytes = 8u << 20;
 __device__ __align__(256) unsigned char g_static_workspace[kStaticWorkspaceBytes];
 
@@ -290,7 +350,7 @@ int static_workspace(int dev, void** out) {
   return VLA_ATTN_OK;
 }
 
-// y = act(x . w^T + bias) (+ res) through one cuBLASLt matmul; argument checks
+// y = act(x . w^T + bias) (+ res) through one launch of the GEMM; argument checks
 // of vla_linear_fwd.
 int linear_impl(const void* x, const void* w, const void* bias, const void* res, void* y, int M,
                 int K, int N, void* workspace, size_t workspace_bytes, void* stream, bool gelu) {
@@ -329,22 +389,22 @@ int linear_impl(const void* x, const void* w, const void* bias, const void* res,
       (workspace_bytes && overlaps(sl, sh, yl, yh)))
     return VLA_ATTN_ERR_MEMORY;
 
-  std::lock_guard<std::mutex> lock(g_lt_mutex);
-  LtPlan* pl = nullptr;
-  rc = lt_plan(dev, M, K, N, bias != nullptr, res != nullptr, gelu, workspace_bytes, &pl);
-  if (rc != VLA_ATTN_OK) return rc;
-  if (bias != nullptr &&
-      cublasLtMatmulDescSetAttribute(pl->op, CUBLASLT_MATMUL_DESC_BIAS_POINTER, &bias,
-                                     sizeof(bias)) != CUBLAS_STATUS_SUCCESS)
-    return VLA_ATTN_ERR_CUDA;
-  const float alpha = 1.0f;
-  const float beta = res != nullptr ? 1.0f : 0.0f;
-  const void* c = res != nullptr ? res : y;
-  if (cublasLtMatmul(g_lt, pl->op, &alpha, w, pl->a, x, pl->b, &beta, c, pl->c, y, pl->c,
-                     &pl->algo, workspace, workspace_bytes,
-                     static_cast<cudaStream_t>(stream)) != CUBLAS_STATUS_SUCCESS)
-    return VLA_ATTN_ERR_CUDA;
-  return VLA_ATTN_OK;
+  const DriverFns& f2 = driver_fns();
+  if (f2.encode == nullptr) return VLA_ATTN_ERR_CUDA;
+  const LinearPlan pl = plan_linear(M, K, N, di.sm_count, workspace_bytes);
+  const int act = gelu ? vla::gemm::kActGelu : vla::gemm::kActNone;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  switch (pl.bn) {
+    case 256:
+      return launch_linear_bn<256>(f2, di, dev, pl, x, w, bias, res, y, M, K, N, act, workspace,
+                                   st);
+    case 128:
+      return launch_linear_bn<128>(f2, di, dev, pl, x, w, bias, res, y, M, K, N, act, workspace,
+                                   st);
+    default:
+      return launch_linear_bn<64>(f2, di, dev, pl, x, w, bias, res, y, M, K, N, act, workspace,
+                                  st);
+  }
 }
 
 }  // namespace
