@@ -461,6 +461,17 @@ def run_configs(args) -> None:
             e1.synchronize()
             warm.append(e0.elapsed_time(e1) * 1e3 / 20)
         del g20
+        # Eager: 200 calls enqueued back to back from Python (argument checks, cached
+        # tensor maps, launch); the host enqueue time per call and the wall time per
+        # call until the stream drains (host-bound when the first is the larger).
+        torch.cuda.synchronize()
+        t0 = time.perf_counter()
+        for _ in range(200):
+            call(c, qkv, out)
+        t1 = time.perf_counter()
+        torch.cuda.synchronize()
+        t2 = time.perf_counter()
+        eager = {"host_enqueue_us": (t1 - t0) / 200 * 1e6, "wall_us": (t2 - t0) / 200 * 1e6}
         # Cold L2: a 256 MB write before each call; the call is enqueued while that
         # write runs, so the events bracket the kernel alone.
         cold = timed(c, qkv, out, min(iters, 50), True)
@@ -471,6 +482,7 @@ def run_configs(args) -> None:
                "roofline_us": t_roof,
                "warm_us": {"median": statistics.median(warm), "p95": _percentile(warm, 0.95)},
                "cold_l2_us": {"median": statistics.median(cold), "p95": _percentile(cold, 0.95)},
+               "eager_us": eager,
                "tflops_warm": flops / statistics.median(warm) / 1e6,
                "frac_warm": t_roof / statistics.median(warm),
                "frac_cold_l2": t_roof / statistics.median(cold)}

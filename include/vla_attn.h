@@ -181,13 +181,14 @@ int vla_layernorm_fwd(const void* x, const void* gamma, const void* beta, void* 
 
 /*
  * Linear layer with bias and optional residual, weights in nn.Linear layout
- * (same page, section 3, CUDA custom operators: cublasLt fused GEMM + bias
- * (+ residual), one launch; the "Pi0 VLA deployment tutorial", section 3.2:
- * the block's qkv linear feeds the attention):
+ * (same page, section 3, CUDA custom operators: GEMM + bias (+ residual) in
+ * one launch; the "Pi0 VLA deployment tutorial", section 3.2: the block's qkv
+ * linear feeds the attention):
  *   y[m,n] = sum_k x[m,k] * w[n,k] + bias[n] + res[m,n]
- * Runs one cuBLASLt matmul (bf16 in, fp32 accumulate, bf16 out, bias in the
- * epilogue, res as C with beta = 1).  For the qkv linear (N = 3 H d), y is the
- * packed [B, tokens, 3, H, d] input of vla_attn_fwd.
+ * One launch of the library's tcgen05 GEMM: bf16 in, fp32 accumulation in
+ * tensor memory, bias and residual added in the fp32 epilogue, one rounding to
+ * bf16 (nearest even).  For the qkv linear (N = 3 H d), y is the packed
+ * [B, tokens, 3, H, d] input of vla_attn_fwd.
  *   x        device, [M, K] bf16 row-major.
  *   w        device, [N, K] bf16 row-major.
  *   bias     device [N] bf16, or NULL (no bias).
@@ -195,12 +196,17 @@ int vla_layernorm_fwd(const void* x, const void* gamma, const void* beta, void* 
  *   y        device, [M, N] bf16 row-major; must not overlap x, w, bias, the
  *            workspace, or res unless it is res.
  *   K, N     multiples of 8.  All pointers 16-byte aligned.
- *   workspace, workspace_bytes  caller-owned device scratch for cuBLASLt
- *            (vla_linear_workspace_bytes() recommended; NULL with 0 allowed);
- *            the library allocates nothing.  Calls that share a workspace
- *            must be ordered on one stream.
- * Returns VLA_ATTN_OK or a negative status (VLA_ATTN_ERR_CUDA if cuBLASLt
- * fails or finds no algorithm).
+ *   workspace, workspace_bytes  caller-owned device scratch (NULL with 0
+ *            allowed).  When the output has too few 128-row tiles to fill the
+ *            SMs, the K range is split and the parts' fp32 partial sums and
+ *            per-tile arrival counters go here (the counters are cleared by a
+ *            memset enqueued before the kernel); a shape is split only if its
+ *            partial sums fit, otherwise it runs unsplit (same result up to
+ *            fp32 summation order).  vla_linear_workspace_bytes() is enough
+ *            for every split the library chooses.  The library allocates
+ *            nothing.  Calls that share a workspace must be ordered on one
+ *            stream.
+ * Returns VLA_ATTN_OK or a negative status.
  */
 int vla_linear_fwd(const void* x, const void* w, const void* bias, const void* res, void* y,
                    int M, int K, int N, void* workspace, size_t workspace_bytes, void* stream);
@@ -222,10 +228,11 @@ int vla_add_layernorm_fwd(const void* x, const void* r, const void* gamma, const
                           void* s, void* y, int M, int W, float eps, void* stream);
 
 /*
- * Linear layer with bias and GELU in one cuBLASLt matmul, the first layer of
- * the ViT MLP (same page, Triton fused kernels: matrix multiply + bias +
- * activation; the activation is GELU in its tanh form,
- * a/2 (1 + tanh(sqrt(2/pi) (a + 0.044715 a^3))), as in SigLIP):
+ * Linear layer with bias and GELU in one launch, the first layer of the ViT
+ * MLP (same page, Triton fused kernels: matrix multiply + bias + activation;
+ * the activation is GELU in its tanh form,
+ * a/2 (1 + tanh(sqrt(2/pi) (a + 0.044715 a^3))), as in SigLIP, evaluated with
+ * the hardware tanh approximation in the GEMM's fp32 epilogue):
  *   y[m,n] = gelu(sum_k x[m,k] * w[n,k] + bias[n])
  *   Layout, alignment, workspace, bias (may be NULL), errors and the
  *   fp32-accumulate, bf16-output arithmetic as vla_linear_fwd; there is no
@@ -238,17 +245,20 @@ int vla_linear_gelu_fwd(const void* x, const void* w, const void* bias, void* y,
 size_t vla_linear_workspace_bytes(void);
 
 /*
- * vla_linear_fwd without a caller workspace and without any allocation: the
- * cuBLASLt workspace is a file-scope device array of
+ * vla_linear_fwd without a caller workspace and without any allocation, for
+ * callers that cannot allocate device memory (for instance code that runs
+ * inside a stream capture, or a runtime that owns all device memory itself):
+ * the split-K scratch is a file-scope device array of
  * vla_linear_static_workspace_bytes() (8 MiB) per device, whose address is
- * looked up once per device with cudaGetSymbolAddress.  cuBLASLt is asked
- * only for algorithms that fit that array; a shape with none is rejected
- * (VLA_ATTN_ERR_CUDA).  Arguments and results otherwise as vla_linear_fwd.
+ * looked up with cudaGetSymbolAddress for each device and context the first
+ * time it is used there.  A shape whose partial sums do not fit it runs
+ * unsplit.  Arguments and results otherwise as vla_linear_fwd.
  *   Calls that overlap on the GPU (on different streams, or from different
  *   host threads without ordering) share the array and race; order them on
- *   one stream.  The first call for a device and shape does the set-up (the
- *   symbol lookup, the cuBLASLt handle and plan): make it before any stream
- *   capture that records later calls.
+ *   one stream.  The array keeps the last call's contents; the arrival
+ *   counters it holds are cleared by each call before its kernel.  The first
+ *   call for a device (and context) does the set-up (the symbol lookup): make
+ *   it before any stream capture that records later calls.
  * The pages have no counterpart of this entry point (a deployment variant of
  * the linear layer, not a step of the method).
  */

@@ -112,6 +112,31 @@ def test_peaked_softmax(sigma, d):
     assert_parity(got, want, f"sigma={sigma} d={d}")
 
 
+@pytest.mark.parametrize("d", [64, 72])
+@pytest.mark.parametrize("boost", [2.0, 6.0, 40.0])
+def test_running_offset_fix_up_positions(d, boost):
+    """Keys whose logits jump far above everything before them, placed in later key blocks
+    at different 16-key chunks (first, middle and last chunk of a block, and the ragged last
+    block): the kernel's weights against the stale running offset fail the chunk check
+    there, and the offset is raised with the chunks already stored, the running sum and O
+    rescaled.  With boost 40 the jump exceeds the fp32 range of 2^x (an overflow to inf
+    that the check must catch).  Every query row is compared with the oracle."""
+    B, N, H = 2, 577, 3
+    bits = si.packed_qkv(B, N, H, d, seed=int(61000 + boost * 10 + d))
+    x = si.bf16_bits_to_f32(bits).copy()
+    u = x[:, :1, 0].copy()                     # one direction per image and head
+    x[:, :, 0] = 0.25 * x[:, :, 0] + u          # every query leans towards u
+    bk = 128 if d == 64 else 112
+    spikes = [bk + 5, 2 * bk + 8 * 7, 3 * bk + bk - 3, N - 1]  # blocks 1-3 and the tail
+    for rank, j in enumerate(spikes):
+        x[:, j, 1] = u[:, 0] * (boost * (rank + 1) / np.sqrt(d))
+    bits = si.f32_to_bf16_bits(x)
+    scale = 1.0 / math.sqrt(d)
+    want = oracle.attention_packed_bf16(bits, scale)
+    got = run_cuda(bits, scale)
+    assert_parity(got, want, f"boost={boost} d={d}")
+
+
 def test_closed_form_inputs_on_gpu():
     """Identical V rows -> O rows equal V; Q = 0 -> O = mean of V (in bf16 precision)."""
     B, N, H, d = 2, 300, 2, 64

@@ -73,26 +73,11 @@ constexpr int kMmaWarp = 0;    // S = Q K^T issuer; also allocates tensor memory
 constexpr int kLoadWarp = 1;   // TMA producer
 constexpr int kPvWarp = 2;     // O += P V issuer
 constexpr int kSoftmaxWarp0 = 4;
-constexpr int kEpilogueWarp0 = 12;
-constexpr int kThreads = 512;
-// Register budgets per warpgroup: the kernel is launched with 128 registers per
-// thread (65,536 for the CTA); the producer / issuer warpgroup and the epilogue
-// warpgroup give registers back so that the two softmax warpgroups can hold a
-// whole S row (128 fp32 values) next to the P chunk they are building.
-// 88 + 56 + 2 x 184 = 512 = 4 x 128.  The host refuses to launch a build whose
-// register count at launch is not kLaunchRegs (an increase that the launch
-// budget cannot cover would wait forever).
-constexpr int kLaunchRegs = 128;
-constexpr uint32_t kRegsIssue = 88;
-constexpr uint32_t kRegsSoftmax = 184;
-constexpr uint32_t kRegsEpilogue = 56;
-static_assert(kRegsIssue + kRegsEpilogue + 2 * kRegsSoftmax <= 4 * kLaunchRegs,
-              "register budgets exceed the launch budget");
+constexpr int kThreads = 384;
 constexpr int kMaxRing = 6;
 constexpr uint32_t kTmemCols = 512;
-constexpr int kNumBarriers = 12 + 4 * kMaxRing + 3 + 6;
+constexpr int kNumBarriers = 12 + 4 * kMaxRing + 3;
 constexpr uint32_t kBarrierRegionBytes = 512;  // barriers + tmem address + abort flag
-constexpr uint32_t kRowSumBytes = 2 * kQRows * 4;  // l of each slot's rows, softmax -> epilogue
 constexpr uint32_t kAlignSlack = 1024;
 constexpr unsigned long long kDrainLimitNs = 100000000ull;
 
@@ -100,8 +85,7 @@ constexpr unsigned long long kDrainLimitNs = 100000000ull;
 enum : int {
   kSiteLoadQ = 1, kSiteLoadK = 2, kSiteLoadV = 3,
   kSiteMmaQ = 11, kSiteMmaK = 12, kSiteMmaV = 13, kSiteMmaP = 14, kSiteMmaFree = 15,
-  kSiteSoftS = 21, kSiteSoftO = 22, kSiteSoftL = 23,
-  kSiteEpiL = 25, kSiteEpiO = 26, kSiteMmaOFree = 16,
+  kSiteSoftS = 21, kSiteSoftO = 22,
   kSiteDrain = 31,
   kSiteTestStall = 41,
 };
@@ -174,7 +158,7 @@ struct AttnParams {
 template <int D>
 __host__ __device__ constexpr uint32_t smem_bytes_for_ring(int ring) {
   return 2u * Geom<D>::kQBytes + 2u * static_cast<uint32_t>(ring) * Geom<D>::kKVStride +
-         kBarrierRegionBytes + kRowSumBytes + kAlignSlack;
+         kBarrierRegionBytes + kAlignSlack;
 }
 
 struct Barriers {
@@ -192,11 +176,6 @@ struct Barriers {
   __device__ uint32_t drain(int i) const { return base + 8u * (12 + 4 * kMaxRing + i); }
   // Never arrived at: the testing hook's wait runs out on it.
   __device__ uint32_t never() const { return base + 8u * (12 + 4 * kMaxRing + 2); }
-  // Softmax -> epilogue: a tile's row sums written (l_full) and read (l_empty).
-  __device__ uint32_t l_full(int s) const { return base + 8u * (12 + 4 * kMaxRing + 3 + s); }
-  __device__ uint32_t l_empty(int s) const { return base + 8u * (12 + 4 * kMaxRing + 5 + s); }
-  // Epilogue -> value issuer: a tile's O read out of tensor memory.
-  __device__ uint32_t o_free(int s) const { return base + 8u * (12 + 4 * kMaxRing + 7 + s); }
 };
 
 // Bounded wait for the phase of `bar` with the given parity, executed by a
@@ -350,7 +329,7 @@ struct RingPos {
 
 // ------------------------------------------------------------ producer
 template <int D>
-__device__ __forceinline__ void load_role(const AttnParams& p, uint32_t sQ, uint32_t sK, uint32_t sV,
+__device__ void load_role(const AttnParams& p, uint32_t sQ, uint32_t sK, uint32_t sV,
                           const Barriers& bar, volatile int* abort_flag) {
   using G = Geom<D>;
   const int R = p.ring;
@@ -440,7 +419,7 @@ __device__ __forceinline__ void load_role(const AttnParams& p, uint32_t sQ, uint
 // Shared-memory descriptors are built once; a K step only moves the start
 // address field (bits [0,14), in 16-byte units), so each step is one add.
 template <int D>
-__device__ __forceinline__ void mma_role(const AttnParams& p, uint32_t tmem, uint32_t sQ, uint32_t sK,
+__device__ void mma_role(const AttnParams& p, uint32_t tmem, uint32_t sQ, uint32_t sK,
                          uint32_t sV, const Barriers& bar, volatile int* abort_flag,
                          bool score_warp) {
   using G = Geom<D>;
@@ -450,7 +429,6 @@ __device__ __forceinline__ void mma_role(const AttnParams& p, uint32_t tmem, uin
   uint32_t nq0 = 0, nq1 = 0;  // q_full phases consumed per Q slot
   uint32_t nf0 = 0, nf1 = 0;  // s_free phases consumed per slot
   uint32_t np0 = 0, np1 = 0;  // p_full phases consumed per slot
-  uint32_t nt0 = 0, nt1 = 0;  // tiles started per slot (o_free phases consumed)
   RingPos pos{0, 0u};         // ring position of the next unit / round's first K/V event
 
   const uint64_t q_desc0 = smem_desc(sQ, 16, 1024, kSwizzle128);
@@ -487,16 +465,6 @@ __device__ __forceinline__ void mma_role(const AttnParams& p, uint32_t tmem, uin
     if (!wait_bounded(bar.s_free(s), nf & 1u, abort_flag, lim, kSiteMmaFree)) return false;
     VLA_TRACE_EVENT(kTrMmaFree, s, 0);
     if (s == 0) ++nf0; else ++nf1;
-    tc_fence_after();
-    return true;
-  };
-  // The first P V of a tile overwrites O: the epilogue must have read the
-  // previous tile's O out of this slot first.
-  auto wait_ofree = [&](int s) -> bool {
-    const uint32_t nt = s == 0 ? nt0 : nt1;
-    if (!wait_bounded(bar.o_free(s), (nt & 1u) ^ 1u, abort_flag, lim, kSiteMmaOFree))
-      return false;
-    if (s == 0) ++nt0; else ++nt1;
     tc_fence_after();
     return true;
   };
@@ -589,7 +557,6 @@ __device__ __forceinline__ void mma_role(const AttnParams& p, uint32_t tmem, uin
         for (int s = 0; ok && s < ns; ++s) {
           if ((!sh || s == 0) && !(ok = wait_v(cur))) break;
           if (!(ok = wait_p(s))) break;
-          if (j == 0 && !(ok = wait_ofree(s))) break;
           values(s, j, cur.slot);
           if (!sh) {
             if (release) commit(bar.v_empty(cur.slot));
@@ -614,108 +581,24 @@ __device__ __forceinline__ void mma_role(const AttnParams& p, uint32_t tmem, uin
 }
 
 // ------------------------------------------------------------ softmax
-constexpr int kPChunk = 8;  // bf16 pairs of P per tensor-memory store
-constexpr int kPHold = 1;   // chunks computed before waiting for the previous P V
-
 struct SoftState {
   float m_run;  // running maximum (raw logits) used for the exponent
   float l_run;  // running sum of weights
 };
 
-// Weights of one key block for one query row against the exponent offset
-// mc = m * c: p = 2^(s c - mc), packed to bf16 pairs and stored to tensor
-// memory in chunks of 16 keys (8 columns).  The first kPHold chunks are
-// computed before waiting for the slot's previous P V (when `wait_pv`), whose
-// completion frees P's columns and makes O safe to rescale.  Returns the fp32 sum of the block's weights in `lsum`,
-// false on abort (before any store).
-template <int NC>
-__device__ __forceinline__ bool exp_block(const float (&x)[NC], float c, float mc, uint32_t tP,
-                                          bool wait_pv, uint32_t pv_parity,
-                                          const AttnParams& p, const Barriers& bar, int s,
-                                          volatile int* abort_flag, float& lsum) {
-  constexpr int kPairs = NC / 2;  // a multiple of 8
-  constexpr int kChunks = kPairs / kPChunk;
-  constexpr int kHold = kPHold < kChunks ? kPHold : kChunks;
-  const uint64_t c2 = f32x2_pack(c, c);
-  const uint64_t nmc2 = f32x2_pack(-mc, -mc);
-  uint64_t acc2[2] = {0ull, 0ull};
-  auto chunk = [&](int ch, uint32_t (&pk)[kPChunk]) {
-#pragma unroll
-    for (int i = 0; i < kPChunk; ++i) {
-      const int k = ch * kPChunk + i;
-      const uint64_t a = f32x2_fma(f32x2_pack(x[2 * k], x[2 * k + 1]), c2, nmc2);
-      float a0, a1;
-      f32x2_unpack(a, a0, a1);
-      const float p0 = ex2_approx(a0);
-      const float p1 = ex2_approx(a1);
-      acc2[i & 1] = f32x2_add(acc2[i & 1], f32x2_pack(p0, p1));
-      pk[i] = pack_bf16x2(p0, p1);
-    }
-  };
-  // The first chunks are held in registers while the previous P V finishes.
-  uint32_t held[kHold][kPChunk];
-#pragma unroll
-  for (int ch = 0; ch < kHold; ++ch) chunk(ch, held[ch]);
-  if (wait_pv) {
-    if (!wait_bounded(bar.o_prog(s), pv_parity, abort_flag, p.wait_limit_ns, kSiteSoftO))
-      return false;
-    tc_fence_after();
-  }
-#pragma unroll
-  for (int ch = 0; ch < kHold; ++ch) tmem_st8(tP + ch * kPChunk, held[ch]);
-#pragma unroll
-  for (int ch = kHold; ch < kChunks; ++ch) {
-    uint32_t pk[kPChunk];
-    chunk(ch, pk);
-    tmem_st8(tP + ch * kPChunk, pk);
-  }
-  float l0, l1, l2, l3;
-  f32x2_unpack(acc2[0], l0, l1);
-  f32x2_unpack(acc2[1], l2, l3);
-  lsum = (l0 + l1) + (l2 + l3);
-  return true;
-}
-
-// Row maximum of a block (NC columns, masked entries already -inf).
-template <int NC>
-__device__ __forceinline__ float row_max(const float (&x)[NC]) {
-  float mx[4] = {x[0], x[1], x[2], x[3]};
-  if constexpr (NC > 4) {
-#pragma unroll
-    for (int i = 4; i + 8 <= NC; i += 8) {
-      mx[0] = fmax3(mx[0], x[i + 0], x[i + 4]);
-      mx[1] = fmax3(mx[1], x[i + 1], x[i + 5]);
-      mx[2] = fmax3(mx[2], x[i + 2], x[i + 6]);
-      mx[3] = fmax3(mx[3], x[i + 3], x[i + 7]);
-    }
-    if constexpr (((NC - 4) % 8) != 0) {
-#pragma unroll
-      for (int i = NC - 4; i < NC; ++i) mx[i & 3] = fmaxf(mx[i & 3], x[i]);
-    }
-  }
-  return fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
-}
-
-// Largest block weight sum accepted against a stale maximum: every weight of
-// the block is at most its sum, so an accepted block has p <= 2^16, and O and
-// l stay far inside the fp32 range (at most 2^30 |v| for 16384 keys).
-constexpr float kStaleSumLimit = 65536.0f;
+// One pair of exponentials in kPolyEvery (0: none) is evaluated on the FMA pipe
+// instead of the special-function unit, the limit of this kernel, sharing its
+// work at the cost of more issued instructions.
+constexpr int kPolyEvery = 16;
 
 // One key block for one query row.  Reads S (NC columns at compile time,
-// nvalid valid at run time) and signals that S has been read.  The first
-// block of a tile sets the running maximum to its row maximum; later blocks
-// exponentiate against the running (stale) maximum without computing their
-// own maximum first, and only if a row's block sum shows a weight above the
-// limit (a maximum that grew by more than about 2^9 / c, or an overflow) does
-// the warp redo the block: that row's maximum is raised to the true one, its
-// sum and O rows rescaled, and the weights recomputed.  The final O / l
-// cancels the common factor, so a stale maximum changes no result beyond
-// rounding.  Returns false on abort.
+// nvalid valid at run time), signals that S has been read, updates the
+// running max / sum, stores P, rescales O when the maximum grew.  Returns
+// false on abort.
 template <int D, int NC>
 __device__ __forceinline__ bool softmax_block(const AttnParams& p, SoftState& st, uint32_t tS,
-                                              uint32_t tO, uint32_t tP, int nvalid, bool first,
-                                              bool wait_pv, uint32_t pv_parity,
-                                              const Barriers& bar, int s,
+                                              uint32_t tO, uint32_t tP, int nvalid, int j,
+                                              const Barriers& bar, int s, uint32_t o_parity,
                                               volatile int* abort_flag, int lane) {
   using G = Geom<D>;
   const float c = p.c;
@@ -735,41 +618,84 @@ __device__ __forceinline__ bool softmax_block(const AttnParams& p, SoftState& st
     for (int i = 0; i < NC; ++i)
       if (i >= nvalid) x[i] = -INFINITY;
   }
-  if (first) st.m_run = row_max<NC>(x);
-  VLA_TRACE_EVENT(kTrSoftMax, s, 0);
-  float lblk;
-  if (!exp_block<NC>(x, c, st.m_run * c, tP, wait_pv, pv_parity, p, bar, s, abort_flag, lblk))
-    return false;
-  const bool bad = !(lblk <= kStaleSumLimit);
-  if (__any_sync(0xffffffffu, bad)) {
-    float alpha = 1.0f;
-    if (bad) {
-      const float m_new = fmaxf(st.m_run, row_max<NC>(x));
-      alpha = ex2_approx((st.m_run - m_new) * c);
-      st.m_run = m_new;
-      st.l_run *= alpha;
+  float mx[4] = {x[0], x[1], x[2], x[3]};
+  if constexpr (NC > 4) {
+#pragma unroll
+    for (int i = 4; i + 8 <= NC; i += 8) {
+      mx[0] = fmax3(mx[0], x[i + 0], x[i + 4]);
+      mx[1] = fmax3(mx[1], x[i + 1], x[i + 5]);
+      mx[2] = fmax3(mx[2], x[i + 2], x[i + 6]);
+      mx[3] = fmax3(mx[3], x[i + 3], x[i + 7]);
     }
-    // P of this block is rewritten in place (its stores are ordered after the
-    // first ones), and the P V that reads it has not been issued yet.
-    tmem_wait_st();
-    (void)exp_block<NC>(x, c, st.m_run * c, tP, false, 0u, p, bar, s, abort_flag, lblk);
-    if (!first) {
-      uint32_t ob[64];
-      tmem_ld64(tO, ob);
+    if constexpr (((NC - 4) % 8) != 0) {
 #pragma unroll
-      for (int i = 0; i < 64; ++i) ob[i] = __float_as_uint(__uint_as_float(ob[i]) * alpha);
-      tmem_st64(tO, ob);
-      if (G::DP > 64) {
-        uint32_t ot[16];
-        tmem_ld16(tO + 64, ot);
-#pragma unroll
-        for (int i = 0; i < 16; ++i) ot[i] = __float_as_uint(__uint_as_float(ot[i]) * alpha);
-        tmem_st16(tO + 64, ot);
-      }
+      for (int i = NC - 4; i < NC; ++i) mx[i & 3] = fmaxf(mx[i & 3], x[i]);
     }
   }
-  VLA_TRACE_EVENT(kTrSoftExp, s, 0);
-  st.l_run += lblk;
+  const float m_blk = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
+  // Keep a stale maximum unless the block's maximum exceeds it by more than 8
+  // in log2 units: the final O / l cancels the common factor, and the weights
+  // stay below 2^8.
+  const bool grow = (m_blk - st.m_run) * c > 8.0f;
+  const bool rescale = __any_sync(0xffffffffu, grow);
+  float alpha = 1.0f;
+  if (rescale) {
+    const float m_new = fmaxf(st.m_run, m_blk);
+    alpha = ex2_approx((st.m_run - m_new) * c);
+    st.m_run = m_new;
+    st.l_run *= alpha;
+  }
+  const float mc = st.m_run * c;
+  VLA_TRACE_EVENT(kTrSoftMax, s, j);
+  // Exponent arguments and running sums in packed fp32 pairs.
+  const uint64_t c2 = f32x2_pack(c, c);
+  const uint64_t nmc2 = f32x2_pack(-mc, -mc);
+  uint64_t acc2[2] = {0ull, 0ull};
+  uint32_t pk[64];
+#pragma unroll
+  for (int i = 0; i < NC / 2; ++i) {
+    const uint64_t a = f32x2_fma(f32x2_pack(x[2 * i], x[2 * i + 1]), c2, nmc2);
+    float p0, p1;
+    if (kPolyEvery > 0 && i % kPolyEvery == kPolyEvery - 1) {
+      exp2_fma_pair(a, p0, p1);  // FMA pipe
+    } else {
+      float a0, a1;
+      f32x2_unpack(a, a0, a1);
+      p0 = ex2_approx(a0);       // special-function unit
+      p1 = ex2_approx(a1);
+    }
+    acc2[i & 1] = f32x2_add(acc2[i & 1], f32x2_pack(p0, p1));
+    pk[i] = pack_bf16x2(p0, p1);
+  }
+  float lsum[4];
+  f32x2_unpack(acc2[0], lsum[0], lsum[1]);
+  f32x2_unpack(acc2[1], lsum[2], lsum[3]);
+#pragma unroll
+  for (int i = NC / 2; i < 64; ++i) pk[i] = 0u;
+  VLA_TRACE_EVENT(kTrSoftExp, s, j);
+  st.l_run += (lsum[0] + lsum[1]) + (lsum[2] + lsum[3]);
+  if (j > 0) {
+    // P V of the previous block must be done before P is overwritten and
+    // before O is touched (this observes every phase of o_prog in order).
+    if (!wait_bounded(bar.o_prog(s), o_parity, abort_flag, p.wait_limit_ns, kSiteSoftO))
+      return false;
+    tc_fence_after();
+  }
+  tmem_st64(tP, pk);
+  if (j > 0 && rescale) {
+    uint32_t ob[64];
+    tmem_ld64(tO, ob);
+#pragma unroll
+    for (int i = 0; i < 64; ++i) ob[i] = __float_as_uint(__uint_as_float(ob[i]) * alpha);
+    tmem_st64(tO, ob);
+    if (G::DP > 64) {
+      uint32_t ot[16];
+      tmem_ld16(tO + 64, ot);
+#pragma unroll
+      for (int i = 0; i < 16; ++i) ot[i] = __float_as_uint(__uint_as_float(ot[i]) * alpha);
+      tmem_st16(tO + 64, ot);
+    }
+  }
   tmem_wait_st();
   return true;
 }
@@ -777,13 +703,11 @@ __device__ __forceinline__ bool softmax_block(const AttnParams& p, SoftState& st
 template <int D>
 __device__ __forceinline__ bool softmax_block_dispatch(const AttnParams& p, SoftState& st,
                                                        uint32_t tS, uint32_t tO, uint32_t tP,
-                                                       int ncols, int nvalid, bool first,
-                                                       bool wait_pv, uint32_t pvp,
-                                                       const Barriers& bar, int s,
+                                                       int ncols, int nvalid, int j,
+                                                       const Barriers& bar, int s, uint32_t op,
                                                        volatile int* abort_flag, int lane) {
-#define VLA_SB(NC)                                                                       \
-  return softmax_block<D, NC>(p, st, tS, tO, tP, nvalid, first, wait_pv, pvp, bar, s, \
-                              abort_flag, lane)
+#define VLA_SB(NC) \
+  return softmax_block<D, NC>(p, st, tS, tO, tP, nvalid, j, bar, s, op, abort_flag, lane)
   if (ncols >= Geom<D>::BK) VLA_SB(Geom<D>::BK);
   switch (ncols) {
     case 112: VLA_SB(112);
@@ -797,12 +721,9 @@ __device__ __forceinline__ bool softmax_block_dispatch(const AttnParams& p, Soft
 #undef VLA_SB
 }
 
-// Softmax warpgroups: one per Q slot, one thread per query row.  After a
-// tile's last block the row sums go to the epilogue warpgroup through shared
-// memory, and the warps go straight on to their next tile.
 template <int D>
-__device__ __forceinline__ void softmax_role(const AttnParams& p, uint32_t tmem, const Barriers& bar,
-                             float* row_sums, volatile int* abort_flag, int warp, int lane) {
+__device__ void softmax_role(const AttnParams& p, uint32_t tmem, const Barriers& bar,
+                             volatile int* abort_flag, int warp, int lane) {
   using G = Geom<D>;
   const int s = (warp - kSoftmaxWarp0) >> 2;  // Q slot of this warpgroup
   const int quad = warp & 3;
@@ -813,8 +734,7 @@ __device__ __forceinline__ void softmax_role(const AttnParams& p, uint32_t tmem,
   const uint32_t tP = tS + G::kColP;
   const int nb = p.num_kblocks;
   uint32_t ns = 0;   // s_full phases consumed
-  uint32_t npv = 0;  // P V issued for this slot so far (o_prog phases to observe)
-  uint32_t nl = 0;   // tiles handed to the epilogue
+  uint32_t npv = 0;  // o_prog phases consumed
   if (p.test_stall) {
     // Testing hook: a wait that nothing completes runs out after the bound,
     // which takes the whole CTA down the error path.
@@ -826,6 +746,7 @@ __device__ __forceinline__ void softmax_role(const AttnParams& p, uint32_t tmem,
     const Round x = next_round(p, cu);
     const bool full = x.nslots == 2;
     if (!full && s == 1) continue;
+    const int tile = x.tile(s);
     SoftState st{-INFINITY, 0.0f};
     for (int j = 0; j < nb; ++j) {
       if (!wait_bounded(bar.s_full(s), ns & 1u, abort_flag, p.wait_limit_ns, kSiteSoftS))
@@ -833,101 +754,51 @@ __device__ __forceinline__ void softmax_role(const AttnParams& p, uint32_t tmem,
       ++ns;
       tc_fence_after();
       VLA_TRACE_EVENT(kTrSoftS, s, j);
-      // Before P is stored: the slot's previous P V (of this tile or the last
-      // one) must be done with P's columns.
       const bool ok = softmax_block_dispatch<D>(
-          p, st, tS, tO, tP, block_cols<G::BK>(p.N, j), min(G::BK, p.N - j * G::BK), j == 0,
-          npv > 0, (npv - 1u) & 1u, bar, s, abort_flag, lane);
+          p, st, tS, tO, tP, block_cols<G::BK>(p.N, j), min(G::BK, p.N - j * G::BK), j, bar, s,
+          (npv + j - 1) & 1u, abort_flag, lane);
       if (!ok) return;
-      ++npv;
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(bar.p_full(s));
       VLA_TRACE_EVENT(kTrSoftP, s, j);
     }
-    // Row sums to the epilogue, once it has read the previous tile's.
-    if (!wait_bounded(bar.l_empty(s), (nl & 1u) ^ 1u, abort_flag, p.wait_limit_ns, kSiteSoftL))
+    // Epilogue: wait for the last P V, then O / l -> bf16, 16-byte stores.
+    if (!wait_bounded(bar.o_prog(s), (npv + nb - 1) & 1u, abort_flag, p.wait_limit_ns,
+                      kSiteSoftO))
       return;
-    ++nl;
-    row_sums[s * kQRows + row_in_tile] = st.l_run;
-    __syncwarp();
-    if (lane == 0) mbar_arrive(bar.l_full(s));
-  }
-}
-
-// ------------------------------------------------------------ epilogue
-// One warpgroup: per tile (in the rounds' slot order), the row sums from the
-// softmax, then O once the tile's last P V is done; O / l -> bf16, 16-byte
-// stores of each valid row (rows >= N and channels >= d are not written).
-// O is read in 16-column pieces, each stored as it arrives; the slot's next
-// first P V may overwrite O as soon as the last piece has been read.
-template <int D>
-__device__ __forceinline__ void epilogue_role(const AttnParams& p, uint32_t tmem, const Barriers& bar,
-                              const float* row_sums, volatile int* abort_flag, int warp,
-                              int lane) {
-  using G = Geom<D>;
-  const int quad = warp & 3;
-  const int row_in_tile = quad * 32 + lane;
-  const uint32_t lane_bits = static_cast<uint32_t>(quad * 32) << 16;
-  const int nb = p.num_kblocks;
-  const unsigned long long lim = p.wait_limit_ns;
-  uint32_t nt0 = 0, nt1 = 0;  // tiles finished per slot
-  constexpr int kPieces = G::DP / 16;  // 4 (d = 64) or 5 (d = 72)
-  for (Cursor cu = cursor_start(); cursor_more(p, cu);) {
-    const Round x = next_round(p, cu);
-    for (int s = 0; s < x.nslots; ++s) {
-      const uint32_t nt = s == 0 ? nt0 : nt1;
-      if (!wait_bounded(bar.l_full(s), nt & 1u, abort_flag, lim, kSiteEpiL)) return;
-      const float l = row_sums[s * kQRows + row_in_tile];
-      __syncwarp();
-      if (lane == 0) mbar_arrive(bar.l_empty(s));
-      // Last P V of this tile: o_prog phase (nt + 1) nb - 1 of the slot.
-      const uint32_t last = (nt + 1u) * static_cast<uint32_t>(nb) - 1u;
-      if (!wait_bounded(bar.o_prog(s), last & 1u, abort_flag, lim, kSiteEpiO)) return;
-      tc_fence_after();
-      if (s == 0) ++nt0; else ++nt1;
-      VLA_TRACE_EVENT(kTrSoftEpi, s, 0);
-      const float inv_l = 1.0f / l;
-      const uint32_t tO = tmem + lane_bits + s * 256 + G::kColO;
-      const int row = x.tile(s) * kQRows + row_in_tile;
+    npv += nb;
+    tc_fence_after();
+    VLA_TRACE_EVENT(kTrSoftEpi, s, 0);
+    const float inv_l = 1.0f / st.l_run;
+    uint32_t ob[64];
+    tmem_ld64(tO, ob);
+    uint32_t ot[16];
+    if (G::DP > 64) tmem_ld16(tO + 64, ot);
+    const int row = tile * kQRows + row_in_tile;
+    if (row < p.N) {
       uint4* dst = reinterpret_cast<uint4*>(
           p.o + ((static_cast<size_t>(x.b(s)) * p.N + row) * p.H + x.h(s)) * D);
-      const bool valid = row < p.N;
 #pragma unroll
-      for (int pc = 0; pc < kPieces; ++pc) {
-        uint32_t ob[16];
-        tmem_ld16(tO + 16 * pc, ob);
+      for (int t = 0; t < D / 8; ++t) {
+        float v[8];
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          if (8 * (2 * pc + h) < D && valid) {
-            float v[8];
-#pragma unroll
-            for (int e = 0; e < 8; ++e) v[e] = __uint_as_float(ob[8 * h + e]) * inv_l;
-            uint4 w;
-            w.x = pack_bf16x2(v[0], v[1]);
-            w.y = pack_bf16x2(v[2], v[3]);
-            w.z = pack_bf16x2(v[4], v[5]);
-            w.w = pack_bf16x2(v[6], v[7]);
-            dst[2 * pc + h] = w;
-          }
+        for (int e = 0; e < 8; ++e) {
+          const int ch = 8 * t + e;
+          v[e] = __uint_as_float(ch < 64 ? ob[ch] : ot[ch - 64]) * inv_l;
         }
+        uint4 w;
+        w.x = pack_bf16x2(v[0], v[1]);
+        w.y = pack_bf16x2(v[2], v[3]);
+        w.z = pack_bf16x2(v[4], v[5]);
+        w.w = pack_bf16x2(v[6], v[7]);
+        dst[t] = w;
       }
-      // All of O has been read: the next tile's first P V may overwrite it.
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(bar.o_free(s));
     }
   }
 }
 
 // ------------------------------------------------------------ kernel
-// Teardown barrier of all kThreads threads (named barrier 1), after each
-// thread's last tensor-memory access.
-__device__ __forceinline__ void teardown_sync() {
-  tc_fence_before();
-  asm volatile("bar.sync 1, %0;" ::"n"(kThreads) : "memory");
-}
-
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_constant__ AttnParams p) {
   using G = Geom<D>;
@@ -941,7 +812,6 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
   uint8_t* bar_generic = smem_raw + (sBar - raw);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_generic + 8 * kNumBarriers);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(bar_generic + 8 * kNumBarriers + 4);
-  float* row_sums = reinterpret_cast<float*>(bar_generic + kBarrierRegionBytes);
   const Barriers bar{sBar};
 
   const int warp = threadIdx.x >> 5;
@@ -955,9 +825,6 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
       mbar_init(bar.s_free(s), 4);
       mbar_init(bar.p_full(s), 4);
       mbar_init(bar.o_prog(s), 1);
-      mbar_init(bar.l_full(s), 4);
-      mbar_init(bar.l_empty(s), 4);
-      mbar_init(bar.o_free(s), 4);
     }
     for (int i = 0; i < kMaxRing; ++i) {
       mbar_init(bar.k_full(i), 1);
@@ -988,37 +855,28 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  // The prologue above (barriers, tensor memory, tensor-map prefetch) may
+  // overlap the previous kernel; global memory is touched only after it.
+  grid_dep_wait();
+  grid_dep_launch();
 
-  // Each warpgroup runs its role under its own register budget and then meets
-  // the others at the teardown barrier inside its own branch (no code after the
-  // branches, so every instruction of a role is compiled against that role's
-  // budget).  Tensor memory is freed once every role has left its loop.
-  if (warp < kSoftmaxWarp0) {
-    regs_dec<kRegsIssue>();
-    if (warp == kLoadWarp) {
-      load_role<D>(p, sQ, sK, sV, bar, abort_flag);
-    } else if (warp == kMmaWarp || warp == kPvWarp) {
-      mma_role<D>(p, tmem, sQ, sK, sV, bar, abort_flag, warp == kMmaWarp);
-    }
+  if (warp == kLoadWarp) {
+    load_role<D>(p, sQ, sK, sV, bar, abort_flag);
     __syncwarp();
-    teardown_sync();
-    VLA_TRACE_END();
-    if (warp == kMmaWarp) {
-      tc_fence_after();
-      tmem_dealloc(tmem, kTmemCols);
-    }
-  } else if (warp < kEpilogueWarp0) {
-    regs_inc<kRegsSoftmax>();
-    softmax_role<D>(p, tmem, bar, row_sums, abort_flag, warp, lane);
+  } else if (warp == kMmaWarp || warp == kPvWarp) {
+    mma_role<D>(p, tmem, sQ, sK, sV, bar, abort_flag, warp == kMmaWarp);
     __syncwarp();
-    teardown_sync();
-    VLA_TRACE_END();
-  } else {
-    regs_dec<kRegsEpilogue>();
-    epilogue_role<D>(p, tmem, bar, row_sums, abort_flag, warp, lane);
+  } else if (warp >= kSoftmaxWarp0) {
+    softmax_role<D>(p, tmem, bar, abort_flag, warp, lane);
     __syncwarp();
-    teardown_sync();
-    VLA_TRACE_END();
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  VLA_TRACE_END();
+  if (warp == kMmaWarp) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
   }
 }
 

@@ -68,6 +68,8 @@ __global__ void __launch_bounds__(256) layernorm_kernel(const __nv_bfloat16* x,
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const long long row = static_cast<long long>(blockIdx.x) * 8 + warp;
+  grid_dep_wait();  // the previous kernel's output is this kernel's input
+  grid_dep_launch();
   if (row >= M) return;
   const __nv_bfloat16* xr = x + row * W;
   float v[NCH][8];
@@ -159,11 +161,21 @@ template <int NCH, bool ADD>
 int launch_layernorm(const void* x, const void* r, const void* gamma, const void* beta, void* s,
                      void* y, long long M, int W, float eps, cudaStream_t stream) {
   const long long blocks = (M + 7) / 8;
-  vla::layernorm_kernel<NCH, ADD><<<static_cast<unsigned>(blocks), 256, 0, stream>>>(
-      static_cast<const __nv_bfloat16*>(x), static_cast<const __nv_bfloat16*>(r),
-      static_cast<const __nv_bfloat16*>(gamma), static_cast<const __nv_bfloat16*>(beta),
-      static_cast<__nv_bfloat16*>(s), static_cast<__nv_bfloat16*>(y), M, W, eps);
-  if (cudaGetLastError() != cudaSuccess) return VLA_ATTN_ERR_CUDA;
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(static_cast<unsigned>(blocks), 1, 1);
+  cfg.blockDim = dim3(256, 1, 1);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  set_dependent_launch(&cfg, attr);
+  if (cudaLaunchKernelEx(&cfg, vla::layernorm_kernel<NCH, ADD>,
+                         static_cast<const __nv_bfloat16*>(x), static_cast<const __nv_bfloat16*>(r),
+                         static_cast<const __nv_bfloat16*>(gamma),
+                         static_cast<const __nv_bfloat16*>(beta), static_cast<__nv_bfloat16*>(s),
+                         static_cast<__nv_bfloat16*>(y), M, W, eps) != cudaSuccess) {
+    (void)cudaGetLastError();
+    return VLA_ATTN_ERR_CUDA;
+  }
   g_launches.fetch_add(1);
   return VLA_ATTN_OK;
 }
@@ -185,12 +197,13 @@ int dispatch_layernorm(const void* x, const void* r, const void* gamma, const vo
 
 // ---------------------------------------------------------------- linear
 // 2-D tensor map of a row-major [rows, K] bf16 matrix, box {64, box_rows},
-// 128-byte swizzle (the K-major operand layout of the GEMM's MMAs).
+// 128-byte swizzle (the K-major operand layout of the GEMM's MMAs, and the
+// epilogue's 64-column staging tiles of y and the residual).
 int encode_2d(const DriverFns& fns, CUtensorMap* map, const void* base, int K, int rows,
               uint32_t box_rows) {
   const cuuint64_t dims[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(rows)};
   const cuuint64_t strides[1] = {static_cast<cuuint64_t>(K) * 2ull};
-  const cuuint32_t box[2] = {static_cast<cuuint32_t>(vla::gemm::kBK), box_rows};
+  const cuuint32_t box[2] = {64u, box_rows};
   const cuuint32_t elem_strides[2] = {1u, 1u};
   const CUresult rc = fns.encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base),
                                  dims, strides, box, elem_strides, CU_TENSOR_MAP_INTERLEAVE_NONE,
@@ -207,10 +220,12 @@ struct LinearPlan {
   size_t workspace_needed = 0;  // partial sums + arrival counters (0 without split K)
 };
 
-// Tile width: the fewest waves of tiles over the SMs weighted by the tile's
-// MMA time (proportional to BN), wider tiles on ties (more reuse per byte
-// loaded).  Split K when the tiles fill at most half the SMs and the caller's
-// workspace holds the partial sums.
+// Tile width: the fewest waves of tiles over the SMs weighted by a tile's cost,
+// its MMA time (proportional to BN) plus its 128-row tile of x (loaded whatever
+// BN is), wider tiles on ties (more reuse per byte loaded).  Split K when the
+// tiles fill at most a quarter of the SMs (with more tiles, adding the parts'
+// partial sums costs more than the split gains) and
+// the caller's workspace holds the partial sums.
 LinearPlan plan_linear(int M, int K, int N, int sm_count, size_t workspace_bytes) {
   LinearPlan pl;
   pl.tiles_m = (M + vla::gemm::kBM - 1) / vla::gemm::kBM;
@@ -218,7 +233,8 @@ LinearPlan plan_linear(int M, int K, int N, int sm_count, size_t workspace_bytes
   long long best = -1;
   for (int bn : {256, 128, 64}) {
     const long long tiles = static_cast<long long>(pl.tiles_m) * ((N + bn - 1) / bn);
-    const long long cost = ((tiles + sm_count - 1) / sm_count) * bn;
+    // Per tile: MMA time ~ BN, plus the 128-row tile of x it loads whatever BN is.
+    const long long cost = ((tiles + sm_count - 1) / sm_count) * (bn + 128);
     if (best < 0 || cost < best) {
       best = cost;
       pl.bn = bn;
@@ -227,7 +243,7 @@ LinearPlan plan_linear(int M, int K, int N, int sm_count, size_t workspace_bytes
   pl.tiles_n = (N + pl.bn - 1) / pl.bn;
   const long long tiles = static_cast<long long>(pl.tiles_m) * pl.tiles_n;
   pl.ksteps_per_split = pl.ksteps;
-  if (2 * tiles <= sm_count && pl.ksteps >= 8) {
+  if (4 * tiles <= sm_count && pl.ksteps >= 8) {
     int splits = static_cast<int>(sm_count / tiles);
     splits = std::min(splits, pl.ksteps / 4);
     splits = std::min(splits, 16);
@@ -259,7 +275,14 @@ int launch_linear_bn(const DriverFns& fns, const DeviceInfo& di, int dev, const 
   if (rc != VLA_ATTN_OK) return rc;
   rc = encode_2d(fns, &prm.tm_b, w, K, N, static_cast<uint32_t>(BN));
   if (rc != VLA_ATTN_OK) return rc;
-  int stages = (di.max_smem_optin - static_cast<int>(vla::gemm::kBarrierBytes + 1024u)) /
+  rc = encode_2d(fns, &prm.tm_y, y, N, M, 32u);
+  if (rc != VLA_ATTN_OK) return rc;
+  if (res != nullptr) {
+    rc = encode_2d(fns, &prm.tm_res, res, N, M, 32u);
+    if (rc != VLA_ATTN_OK) return rc;
+  }
+  int stages = (di.max_smem_optin - static_cast<int>(vla::gemm::kStagingBytes +
+                                                     vla::gemm::kBarrierBytes + 1024u)) /
                static_cast<int>(G::kStageBytes);
   if (stages > vla::gemm::kMaxStages) stages = vla::gemm::kMaxStages;
   if (stages < 2) return VLA_ATTN_ERR_DEVICE;
@@ -308,6 +331,9 @@ int launch_linear_bn(const DriverFns& fns, const DeviceInfo& di, int dev, const 
   cfg.blockDim = dim3(vla::gemm::kThreads, 1, 1);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;
+  // A split launch follows the memset of its counters: ordinary stream order.
+  cudaLaunchAttribute attr[1];
+  if (pl.splits == 1) set_dependent_launch(&cfg, attr);
   if (cudaLaunchKernelEx(&cfg, vla::gemm::linear_kernel<BN>, prm) != cudaSuccess) {
     (void)cudaGetLastError();
     return VLA_ATTN_ERR_CUDA;

@@ -25,7 +25,8 @@
 //               columns), so the epilogue of one tile overlaps the next
 //               tile's MMAs.
 //   warps 4-7   epilogue: one thread per output row (= tensor-memory lane),
-//               32 columns per tensor-memory load, 16-byte stores.
+//               64 columns at a time staged in shared memory (the residual
+//               brought in by a TMA load) and written by TMA stores.
 //   warps 2-3   idle.
 // Split K: with few output tiles the K range is cut into `splits` parts; each
 // part's CTA writes fp32 partial sums to the caller's workspace, and for each
@@ -56,7 +57,12 @@ constexpr int kLoadWarp = 0;
 constexpr int kMmaWarp = 1;
 constexpr int kEpiWarp0 = 4;
 constexpr int kMaxStages = 8;
-constexpr uint32_t kBarrierBytes = 256;  // 2 kMaxStages + 4 + 2 barriers, tmem address, flags
+constexpr uint32_t kBarrierBytes = 512;  // 2 kMaxStages + 6 + 8 barriers, tmem address, flags
+// Output staging of the epilogue: per epilogue warp two buffers of 32 rows x 64
+// columns of bf16 (4 KB, 128-byte swizzle) that TMA stores to y (and that a TMA
+// load fills with the residual first).
+constexpr uint32_t kStageOutBytes = 32 * 128;
+constexpr uint32_t kStagingBytes = 4 * 2 * kStageOutBytes;
 
 enum : int { kActNone = 0, kActGelu = 1 };
 
@@ -68,6 +74,8 @@ enum : int {
 struct GemmParams {
   CUtensorMap tm_a;              // x [M, K] bf16, box {64, 128}
   CUtensorMap tm_b;              // w [N, K] bf16, box {64, BN}
+  CUtensorMap tm_y;              // y [M, N] bf16, box {64, 32} (epilogue stores)
+  CUtensorMap tm_res;            // res [M, N] bf16, box {64, 32} (when res is given)
   const __nv_bfloat16* bias;     // [N] or null
   const __nv_bfloat16* res;      // [M, N] or null (may be y itself)
   __nv_bfloat16* y;              // [M, N]
@@ -96,7 +104,8 @@ struct GemmGeom {
 
 template <int BN>
 __host__ __device__ constexpr uint32_t gemm_smem_bytes(int stages) {
-  return static_cast<uint32_t>(stages) * GemmGeom<BN>::kStageBytes + kBarrierBytes + 1024u;
+  return static_cast<uint32_t>(stages) * GemmGeom<BN>::kStageBytes + kStagingBytes +
+         kBarrierBytes + 1024u;
 }
 
 struct GemmBarriers {
@@ -106,7 +115,35 @@ struct GemmBarriers {
   __device__ uint32_t acc_full(int b) const { return base + 8u * (2 * kMaxStages + b); }
   __device__ uint32_t acc_empty(int b) const { return base + 8u * (2 * kMaxStages + 2 + b); }
   __device__ uint32_t drain(int i) const { return base + 8u * (2 * kMaxStages + 4 + i); }
+  // Residual tile landed in staging buffer b of epilogue warp e.
+  __device__ uint32_t res_full(int e, int b) const {
+    return base + 8u * (2 * kMaxStages + 6 + 2 * e + b);
+  }
 };
+
+// Tiled 2-D store of a shared-memory box to global memory (bulk group), and
+// the waits on this thread's bulk groups: until at most N of them still read
+// shared memory, and until all have completed.
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, uint32_t src, int c0, int c1) {
+  asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%1, %2}], [%3];" ::"l"(
+                   reinterpret_cast<uint64_t>(map)),
+               "r"(c0), "r"(c1), "r"(src)
+               : "memory");
+}
+__device__ __forceinline__ void bulk_commit() {
+  asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+template <int N>
+__device__ __forceinline__ void bulk_wait_read() {
+  asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(N) : "memory");
+}
+__device__ __forceinline__ void bulk_wait_all() {
+  asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+}
+// Makes this thread's shared-memory writes visible to the TMA unit.
+__device__ __forceinline__ void fence_async_shared() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
 
 // 2-D tiled load of one box into shared memory, completing on `bar`.
 __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, uint32_t bar,
@@ -118,16 +155,19 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map
       : "memory");
 }
 
-// Work item w -> output tile and K part.  Tiles are walked N-fastest within an
-// M row so that the CTAs running at one time share the rows of x they read
-// (w, at most a few MB for these layers, stays in L2).
+// The k-th work item of this CTA -> output tile and K part; false when the CTA
+// has no k-th item.  Items w = blockIdx.x + k G of the list ordered split, then
+// M row, then N tile: the CTAs running at one time cover a few rows of tiles,
+// all N tiles of each, so a row block of x is read from DRAM about once and
+// w (at most a few MB for these layers) stays in L2.
 struct Work {
   int mt, nt, split;
   int k0, k1;  // k-steps [k0, k1)
 };
 
-__device__ __forceinline__ Work work_item(const GemmParams& p, int w) {
-  Work r;
+__device__ __forceinline__ bool work_at(const GemmParams& p, int k, Work& r) {
+  const int w = static_cast<int>(blockIdx.x) + k * static_cast<int>(gridDim.x);
+  if (w >= p.num_work) return false;
   const int tiles = p.tiles_m * p.tiles_n;
   r.split = w / tiles;
   const int t = w - r.split * tiles;
@@ -135,7 +175,7 @@ __device__ __forceinline__ Work work_item(const GemmParams& p, int w) {
   r.nt = t - r.mt * p.tiles_n;
   r.k0 = r.split * p.ksteps_per_split;
   r.k1 = min(p.ksteps, r.k0 + p.ksteps_per_split);
-  return r;
+  return true;
 }
 
 template <int BN>
@@ -147,8 +187,8 @@ __device__ __forceinline__ void gemm_load_role(const GemmParams& p, uint32_t sba
   uint32_t phase = 0;
   uint32_t issued = 0;
   bool ok = true;
-  for (int w = blockIdx.x; ok && w < p.num_work; w += gridDim.x) {
-    const Work wk = work_item(p, w);
+  Work wk;
+  for (int k = 0; ok && work_at(p, k, wk); ++k) {
     for (int ks = wk.k0; ks < wk.k1; ++ks) {
       if (!wait_bounded(bar.empty(stage), phase ^ 1u, abort_flag, p.wait_limit_ns, kSiteLoad)) {
         ok = false;
@@ -188,9 +228,8 @@ __device__ __forceinline__ void gemm_mma_role(const GemmParams& p, uint32_t tmem
   int stage = 0;
   uint32_t phase = 0;
   bool ok = true;
-  int i = 0;  // work items of this CTA
-  for (int w = blockIdx.x; ok && w < p.num_work; w += gridDim.x, ++i) {
-    const Work wk = work_item(p, w);
+  Work wk;
+  for (int i = 0; ok && work_at(p, i, wk); ++i) {  // i: work items of this CTA
     const int buf = i & 1;
     // The epilogue must have read this accumulator's previous tile.
     if (!wait_bounded(bar.acc_empty(buf), ((i >> 1) & 1) ^ 1, abort_flag, p.wait_limit_ns,
@@ -277,18 +316,57 @@ __device__ __forceinline__ void store8(const GemmParams& p, const float (&acc)[8
   *reinterpret_cast<uint4*>(p.y + off) = o;
 }
 
+// Epilogue of 8 consecutive columns n.. of one row from fp32 accumulators:
+// (+ bias) -> act (+ the residual's 8 bf16 values) -> 4 packed bf16 pairs.
+__device__ __forceinline__ uint4 epi8(const GemmParams& p, const uint32_t* acc, int n,
+                                      const uint4* res8) {
+  float v[8];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) v[e] = __uint_as_float(acc[e]);
+  if (p.bias != nullptr && n < p.N) {
+    const uint4 bb = *reinterpret_cast<const uint4*>(p.bias + n);
+    const uint32_t bw[4] = {bb.x, bb.y, bb.z, bb.w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      v[2 * e] += __uint_as_float(bw[e] << 16);
+      v[2 * e + 1] += __uint_as_float(bw[e] & 0xFFFF0000u);
+    }
+  }
+  if (p.act == kActGelu) {
+#pragma unroll
+    for (int e = 0; e < 8; ++e) v[e] = gelu_tanh(v[e]);
+  }
+  if (res8 != nullptr) {
+    const uint32_t rw[4] = {res8->x, res8->y, res8->z, res8->w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      v[2 * e] += __uint_as_float(rw[e] << 16);
+      v[2 * e + 1] += __uint_as_float(rw[e] & 0xFFFF0000u);
+    }
+  }
+  uint4 o;
+  o.x = pack_bf16x2(v[0], v[1]);
+  o.y = pack_bf16x2(v[2], v[3]);
+  o.z = pack_bf16x2(v[4], v[5]);
+  o.w = pack_bf16x2(v[6], v[7]);
+  return o;
+}
+
 template <int BN>
 __device__ __forceinline__ void gemm_epilogue_role(const GemmParams& p, uint32_t tmem,
                                                    const GemmBarriers& bar,
-                                                   volatile int* abort_flag, int warp, int lane) {
+                                                   volatile int* abort_flag, int warp, int lane,
+                                                   uint32_t staging) {
   const int quad = warp & 3;
+  const int ew = warp - kEpiWarp0;  // epilogue warp 0..3
+  const uint32_t stg = staging + static_cast<uint32_t>(ew) * 2u * kStageOutBytes;
+  uint32_t chunks_done = 0;         // staged chunks of this warp (alternating buffers)
   const int r_in = quad * 32 + lane;
   const uint32_t lane_bits = static_cast<uint32_t>(quad * 32) << 16;
   const size_t tile_elems = static_cast<size_t>(kBM) * BN;
   const int tiles = p.tiles_m * p.tiles_n;
-  int i = 0;
-  for (int w = blockIdx.x; w < p.num_work; w += gridDim.x, ++i) {
-    const Work wk = work_item(p, w);
+  Work wk;
+  for (int i = 0; work_at(p, i, wk); ++i) {
     const int buf = i & 1;
     if (!wait_bounded(bar.acc_full(buf), (i >> 1) & 1, abort_flag, p.wait_limit_ns, kSiteEpi))
       return;
@@ -298,7 +376,7 @@ __device__ __forceinline__ void gemm_epilogue_role(const GemmParams& p, uint32_t
     const int n_base = wk.nt * BN;
     if (p.splits > 1) {
       // Partial sums of this K part to the workspace (row-major within the tile).
-      const int tile = w - wk.split * tiles;
+      const int tile = wk.mt * p.tiles_n + wk.nt;
       float* part = p.partial + (static_cast<size_t>(wk.split) * tiles + tile) * tile_elems +
                     static_cast<size_t>(r_in) * BN;
 #pragma unroll 1
@@ -322,49 +400,108 @@ __device__ __forceinline__ void gemm_epilogue_role(const GemmParams& p, uint32_t
       prev = __shfl_sync(0xffffffffu, prev, 0);
       if (prev != static_cast<unsigned int>(p.splits - 1)) continue;
       __threadfence();
-      if (row < p.M) {
-        const float* base = p.partial + static_cast<size_t>(tile) * tile_elems +
-                            static_cast<size_t>(r_in) * BN;
+      // Coalesced: BN / 8 lanes cover one row (8 columns each), 32 / (BN / 8) rows per
+      // pass; every split's partial sums of a lane are loaded before they are added.
+      constexpr int kLanesPerRow = BN / 8 < 32 ? BN / 8 : 32;
+      constexpr int kRowsPerPass = 32 / kLanesPerRow;
+      constexpr int kColPasses = BN / 8 / kLanesPerRow;  // 1, except 256-wide tiles: 1
+      const int col = (lane % kLanesPerRow) * 8;
+      const float* tile_part = p.partial + static_cast<size_t>(tile) * tile_elems;
+      const size_t split_stride = static_cast<size_t>(tiles) * tile_elems;
+      // Four passes at a time: all their partial-sum loads are in flight together.
+      constexpr int kPasses = 32 / kRowsPerPass;
+      constexpr int kGroup = kPasses < 4 ? kPasses : 4;
+      static_assert(kColPasses == 1, "one column pass per row");
 #pragma unroll 1
-        for (int g = 0; g < BN / 8; ++g) {
-          const int n = n_base + 8 * g;
-          if (n >= p.N) break;
-          float acc[8];
+      for (int pg = 0; pg < kPasses; pg += kGroup) {
+        float acc[kGroup][8];
 #pragma unroll
-          for (int e = 0; e < 8; ++e) acc[e] = 0.0f;
-          for (int sp = 0; sp < p.splits; ++sp) {
-            const float4* src = reinterpret_cast<const float4*>(
-                base + static_cast<size_t>(sp) * tiles * tile_elems + 8 * g);
-            const float4 u = __ldcg(src), v = __ldcg(src + 1);
-            acc[0] += u.x; acc[1] += u.y; acc[2] += u.z; acc[3] += u.w;
-            acc[4] += v.x; acc[5] += v.y; acc[6] += v.z; acc[7] += v.w;
+        for (int g = 0; g < kGroup; ++g)
+#pragma unroll
+          for (int e = 0; e < 8; ++e) acc[g][e] = 0.0f;
+#pragma unroll 2
+        for (int sp = 0; sp < p.splits; ++sp) {
+          float4 u[kGroup], v[kGroup];
+#pragma unroll
+          for (int g = 0; g < kGroup; ++g) {
+            const int rl = quad * 32 + (pg + g) * kRowsPerPass + lane / kLanesPerRow;
+            const float4* q = reinterpret_cast<const float4*>(
+                tile_part + sp * split_stride + static_cast<size_t>(rl) * BN + col);
+            u[g] = __ldcg(q);
+            v[g] = __ldcg(q + 1);
           }
-          store8(p, acc, row, n);
+#pragma unroll
+          for (int g = 0; g < kGroup; ++g) {
+            acc[g][0] += u[g].x; acc[g][1] += u[g].y; acc[g][2] += u[g].z; acc[g][3] += u[g].w;
+            acc[g][4] += v[g].x; acc[g][5] += v[g].y; acc[g][6] += v[g].z; acc[g][7] += v[g].w;
+          }
+        }
+#pragma unroll
+        for (int g = 0; g < kGroup; ++g) {
+          const int rl = quad * 32 + (pg + g) * kRowsPerPass + lane / kLanesPerRow;
+          const int grow = wk.mt * kBM + rl;
+          const int n = n_base + col;
+          if (grow < p.M && n < p.N) store8(p, acc[g], grow, n);
         }
       }
       continue;
     }
+    // 64 columns at a time: the residual (if any) arrives in a staging buffer by
+    // TMA, each thread writes its row's 64 results into the buffer (128-byte
+    // swizzle: 16-byte piece j of row r at piece j ^ (r % 8)), and one TMA
+    // store writes the 32 x 64 box; rows >= M and columns >= N are clipped.
+    const int row0 = wk.mt * kBM + quad * 32;
 #pragma unroll 1
-    for (int c = 0; c < BN / 32; ++c) {
-      uint32_t a[32];
-      tmem_ld32(t + 32 * c, a);
-      if (row < p.M) {
-#pragma unroll
-        for (int g = 0; g < 4; ++g) {
-          const int n = n_base + 32 * c + 8 * g;
-          if (n < p.N) {
-            float acc[8];
-#pragma unroll
-            for (int e = 0; e < 8; ++e) acc[e] = __uint_as_float(a[8 * g + e]);
-            store8(p, acc, row, n);
-          }
+    for (int c = 0; c < BN / 64; ++c) {
+      const int bsel = static_cast<int>(chunks_done & 1u);
+      const uint32_t buf_s = stg + static_cast<uint32_t>(bsel) * kStageOutBytes;
+      const int n0 = n_base + 64 * c;
+      // The store that last read this buffer must be done reading it.
+      if (lane == 0) bulk_wait_read<1>();
+      __syncwarp();
+      if (p.res != nullptr) {
+        const uint32_t rb = bar.res_full(ew, bsel);
+        if (lane == 0) {
+          mbar_arrive_expect_tx(rb, kStageOutBytes);
+          tma_load_2d(buf_s, &p.tm_res, rb, n0, row0);
         }
+        if (!wait_bounded(rb, (chunks_done >> 1) & 1u, abort_flag, p.wait_limit_ns, kSiteEpi))
+          return;
       }
+      uint32_t a[64];
+      tmem_ld32(t + 64 * c, reinterpret_cast<uint32_t(&)[32]>(a[0]));
+      tmem_ld32(t + 64 * c + 32, reinterpret_cast<uint32_t(&)[32]>(a[32]));
+      const uint32_t row_s = buf_s + static_cast<uint32_t>(lane) * 128u;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const uint32_t piece = row_s + static_cast<uint32_t>((j ^ (lane & 7)) * 16);
+        uint4 r8;
+        if (p.res != nullptr) {
+          asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                       : "=r"(r8.x), "=r"(r8.y), "=r"(r8.z), "=r"(r8.w)
+                       : "r"(piece));
+        }
+        const uint4 o = epi8(p, a + 8 * j, n0 + 8 * j, p.res != nullptr ? &r8 : nullptr);
+        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(piece), "r"(o.x),
+                     "r"(o.y), "r"(o.z), "r"(o.w)
+                     : "memory");
+      }
+      fence_async_shared();
+      __syncwarp();
+      if (lane == 0) {
+        tma_store_2d(&p.tm_y, buf_s, n0, row0);
+        bulk_commit();
+      }
+      ++chunks_done;
     }
+    (void)row;
     tc_fence_before();
     __syncwarp();
     if (lane == 0) mbar_arrive(bar.acc_empty(buf));
   }
+  // Every TMA store of this warp must have finished before the CTA exits.
+  if (lane == 0) bulk_wait_all();
+  __syncwarp();
 }
 
 __device__ __forceinline__ void gemm_teardown_sync() {
@@ -378,7 +515,8 @@ __global__ void __launch_bounds__(kThreads, 1) linear_kernel(const __grid_consta
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t sbase = (raw + 1023u) & ~1023u;
-  const uint32_t sbar = sbase + static_cast<uint32_t>(p.stages) * G::kStageBytes;
+  const uint32_t staging = sbase + static_cast<uint32_t>(p.stages) * G::kStageBytes;
+  const uint32_t sbar = staging + kStagingBytes;
   uint8_t* bar_generic = smem_raw + (sbar - raw);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_generic + 8 * (2 * kMaxStages + 6));
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
@@ -395,6 +533,7 @@ __global__ void __launch_bounds__(kThreads, 1) linear_kernel(const __grid_consta
       mbar_init(bar.acc_full(b), 1);
       mbar_init(bar.acc_empty(b), 4);
       mbar_init(bar.drain(b), 1);
+      for (int e = 0; e < 4; ++e) mbar_init(bar.res_full(e, b), 1);
     }
     *abort_flag = 0;
     fence_mbar_init();
@@ -402,6 +541,8 @@ __global__ void __launch_bounds__(kThreads, 1) linear_kernel(const __grid_consta
   if (warp == kLoadWarp && lane == 0) {
     prefetch_tmap(&p.tm_a);
     prefetch_tmap(&p.tm_b);
+    prefetch_tmap(&p.tm_y);
+    if (p.res != nullptr) prefetch_tmap(&p.tm_res);
   }
   if (warp == kMmaWarp) {
     tmem_alloc(smem_u32(tmem_slot), G::kTmemCols);
@@ -411,13 +552,17 @@ __global__ void __launch_bounds__(kThreads, 1) linear_kernel(const __grid_consta
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  // The prologue may overlap the previous kernel (programmatic dependent
+  // launch); global memory is touched only after this wait.
+  grid_dep_wait();
+  grid_dep_launch();
 
   if (warp == kLoadWarp) {
     gemm_load_role<BN>(p, sbase, bar, abort_flag);
   } else if (warp == kMmaWarp) {
     gemm_mma_role<BN>(p, tmem, sbase, bar, abort_flag);
   } else if (warp >= kEpiWarp0) {
-    gemm_epilogue_role<BN>(p, tmem, bar, abort_flag, warp, lane);
+    gemm_epilogue_role<BN>(p, tmem, bar, abort_flag, warp, lane, staging);
   }
   __syncwarp();
   gemm_teardown_sync();

@@ -149,26 +149,22 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
 
 #define VLA_R32(i) VLA_R8(i), VLA_R8(i + 8), VLA_R8(i + 16), VLA_R8(i + 24)
 
-// 128 consecutive fp32 columns of this thread's lane: two 64-column loads and
-// one completion wait in the same asm block (an instruction with 128
-// destination registers would not fit a kernel compiled for 128 registers per
-// thread, although the calling warp may hold more after setmaxnreg).
+// 128 consecutive fp32 columns of this thread's lane in one instruction.
 __device__ __forceinline__ void tmem_ld128(uint32_t taddr, uint32_t (&r)[128]) {
   asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x64.b32 "
+      "tcgen05.ld.sync.aligned.32x32b.x128.b32 "
       "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
       "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, "
       "%32, %33, %34, %35, %36, %37, %38, %39, %40, %41, %42, %43, %44, %45, %46, %47, "
-      "%48, %49, %50, %51, %52, %53, %54, %55, %56, %57, %58, %59, %60, %61, %62, %63}, [%128];\n\t"
-      "tcgen05.ld.sync.aligned.32x32b.x64.b32 "
-      "{%64, %65, %66, %67, %68, %69, %70, %71, %72, %73, %74, %75, %76, %77, %78, %79, "
+      "%48, %49, %50, %51, %52, %53, %54, %55, %56, %57, %58, %59, %60, %61, %62, %63, "
+      "%64, %65, %66, %67, %68, %69, %70, %71, %72, %73, %74, %75, %76, %77, %78, %79, "
       "%80, %81, %82, %83, %84, %85, %86, %87, %88, %89, %90, %91, %92, %93, %94, %95, "
       "%96, %97, %98, %99, %100, %101, %102, %103, %104, %105, %106, %107, %108, %109, %110, "
       "%111, %112, %113, %114, %115, %116, %117, %118, %119, %120, %121, %122, %123, %124, "
-      "%125, %126, %127}, [%129];\n\t"
+      "%125, %126, %127}, [%128];\n\t"
       "tcgen05.wait::ld.sync.aligned;"
       : VLA_R32(0), VLA_R32(32), VLA_R32(64), VLA_R32(96)
-      : "r"(taddr), "r"(taddr + 64u)
+      : "r"(taddr)
       : "memory");
 }
 
@@ -221,14 +217,6 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16
       : "memory");
 }
 
-__device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t (&r)[8]) {
-  asm volatile(
-      "tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], "
-      "{%1, %2, %3, %4, %5, %6, %7, %8};" ::"r"(taddr),
-      VLA_S8(0)
-      : "memory");
-}
-
 __device__ __forceinline__ void tmem_wait_st() {
   asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
@@ -258,16 +246,17 @@ __host__ __device__ constexpr uint32_t idesc_bf16_m128(uint32_t n, uint32_t b_mn
          ((128u >> 4) << 24);
 }
 
-// Per-warpgroup register budgets (executed by all warps of a warpgroup).  An
-// increase draws on the registers the CTA was launched with, so the budgets of
-// all warpgroups must sum to at most the launch budget.
-template <uint32_t R>
-__device__ __forceinline__ void regs_dec() {
-  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(R));
+// Programmatic dependent launch.  A kernel launched with programmatic stream
+// serialization may start while the kernel before it on the stream is still
+// running; `grid_dep_wait` blocks until that kernel has completed and its
+// memory is visible (a no-op for a kernel launched without the attribute), so
+// it must precede every global-memory access.  `grid_dep_launch` lets the next
+// such kernel start once every CTA of this grid has executed it or exited.
+__device__ __forceinline__ void grid_dep_wait() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
 }
-template <uint32_t R>
-__device__ __forceinline__ void regs_inc() {
-  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(R));
+__device__ __forceinline__ void grid_dep_launch() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
 // ------------------------------------------------------------------- warp
@@ -307,6 +296,32 @@ __device__ __forceinline__ uint64_t f32x2_add(uint64_t a, uint64_t b) {
   uint64_t d;
   asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
   return d;
+}
+
+// 2^a for a packed pair on the FMA pipe instead of the special-function unit:
+// a clamped at -126, n = round(a) by adding 1.5 * 2^23 (n lands in the low
+// mantissa bits of t), f = a - n in [-1/2, 1/2], 2^f by a cubic in Horner
+// form (coefficients from a minimax fit of 2^f on [-1/2, 1/2], relative
+// error below 7.5e-5), and n added to the exponent field as an integer
+// (t's bits shifted left by 23 are n << 23 modulo 2^32).  For arguments
+// above 127 the result is not 2^a; callers keep a <= 8.
+__device__ __forceinline__ void exp2_fma_pair(uint64_t a, float& y0, float& y1) {
+  float a0, a1;
+  f32x2_unpack(a, a0, a1);
+  const uint64_t ac = f32x2_pack(fmaxf(a0, -126.0f), fmaxf(a1, -126.0f));
+  const uint64_t magic = f32x2_pack(12582912.0f, 12582912.0f);
+  const uint64_t t = f32x2_add(ac, magic);
+  const uint64_t r = f32x2_add(t, f32x2_pack(-12582912.0f, -12582912.0f));
+  const uint64_t f = f32x2_fma(r, f32x2_pack(-1.0f, -1.0f), ac);
+  uint64_t q = f32x2_fma(f32x2_pack(0.05517167f, 0.05517167f), f,
+                         f32x2_pack(0.24261113f, 0.24261113f));
+  q = f32x2_fma(q, f, f32x2_pack(0.69326097f, 0.69326097f));
+  q = f32x2_fma(q, f, f32x2_pack(0.99992806f, 0.99992806f));
+  float q0, q1, t0, t1;
+  f32x2_unpack(q, q0, q1);
+  f32x2_unpack(t, t0, t1);
+  y0 = __uint_as_float(__float_as_uint(q0) + (__float_as_uint(t0) << 23));
+  y1 = __uint_as_float(__float_as_uint(q1) + (__float_as_uint(t1) << 23));
 }
 
 __device__ __forceinline__ float fmax3(float a, float b, float c) {

@@ -96,6 +96,17 @@ int device_info(int dev, DeviceInfo* out) {
   return di.supported ? VLA_ATTN_OK : VLA_ATTN_ERR_DEVICE;
 }
 
+// Programmatic dependent launch for a kernel launch: the kernel may start (and
+// run its prologue) while the previous kernel on the stream finishes; every
+// kernel of this library waits for that kernel (griddepcontrol.wait) before it
+// touches global memory, so stream order is kept for all data.
+void set_dependent_launch(cudaLaunchConfig_t* cfg, cudaLaunchAttribute (&attr)[1]) {
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg->attrs = attr;
+  cfg->numAttrs = 1;
+}
+
 // Copy-out stream and fork / join events of the pipelined host-buffer entry,
 // one set per device, created on first use (guarded by g_pipe_mutex, which
 // the caller holds for the whole enqueue sequence).
@@ -298,13 +309,11 @@ int launch(const void* q, void* o, int B, int N, int H, float scale, cudaStream_
   if (rc != VLA_ATTN_OK) return rc;
   const int nb = (N + G::BK - 1) / G::BK;
   const int nq = (N + vla::kQRows - 1) / vla::kQRows;
-  // The warpgroups re-divide the registers the CTA is launched with (setmaxnreg);
-  // that division assumes exactly kLaunchRegs per thread at launch.
   const KernelAttrs& ka = kernel_attrs<D>();
-  if (!ka.ok || ka.regs != vla::kLaunchRegs) return VLA_ATTN_ERR_CUDA;
+  if (!ka.ok) return VLA_ATTN_ERR_CUDA;
   const int max_smem = di.max_smem_optin - ka.static_smem;
   int ring = (max_smem - static_cast<int>(2 * G::kQBytes + vla::kBarrierRegionBytes +
-                                          vla::kRowSumBytes + vla::kAlignSlack)) /
+                                          vla::kAlignSlack)) /
              static_cast<int>(2 * G::kKVStride);
   if (ring > vla::kMaxRing) ring = vla::kMaxRing;
   if (ring < 2) return VLA_ATTN_ERR_DEVICE;
@@ -346,8 +355,8 @@ int launch(const void* q, void* o, int B, int N, int H, float scale, cudaStream_
   cfg.blockDim = dim3(vla::kThreads, 1, 1);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;
-  cfg.attrs = nullptr;
-  cfg.numAttrs = 0;
+  cudaLaunchAttribute attr[1];
+  set_dependent_launch(&cfg, attr);
   if (cudaLaunchKernelEx(&cfg, vla::attn_fwd_kernel<D>, prm) != cudaSuccess) {
     (void)cudaGetLastError();
     return VLA_ATTN_ERR_CUDA;
