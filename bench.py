@@ -7,7 +7,8 @@ batch.  Prints ONE JSON line (rank 0).
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
   python bench.py --configs     # per-config report (one JSON line per item, 1 GPU)
-  python bench.py --block       # LayerNorm / linear layers and the attention half-block
+  python bench.py --block       # LayerNorm / linear layers, whole encoder layers and encoders
+  python bench.py --linear M,K,N   # one linear layer of that shape
 
 Under torchrun every rank runs the same per-GPU batch on its own GPU (weak
 scaling, no collective on the data path); the elapsed time is the max over
@@ -679,6 +680,47 @@ def run_block(args) -> None:
         torch.cuda.empty_cache()
 
 
+def run_linear(args) -> None:
+    """One linear layer y = x w^T + bias on an (M, K, N) shape, seeded bf16 operands: five
+    warm calls, then the median of 20 CUDA-event timed calls (one JSON line).  Small enough
+    to run under ncu (the GEMM's profile)."""
+    import math as _m
+
+    import torch
+
+    import vit_self_attention_b200 as vab
+
+    M, K, N = (int(v) for v in args.linear.split(","))
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+
+    def t_(shape, std, seed):
+        b = si.normal_bf16(seed, shape, 0.0, std)
+        return torch.from_numpy(b.view(np.int16)).to(dev).view(torch.bfloat16)
+
+    x, w, b = t_((M, K), 1.0, 21), t_((N, K), 1.0 / _m.sqrt(K), 22), t_((N,), 0.1, 23)
+    y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+    ws = torch.empty(vab.vla_linear_workspace_bytes(), dtype=torch.uint8, device=dev)
+    for _ in range(5):
+        vab.linear(x, w, b, out=y, workspace=ws)
+    torch.cuda.synchronize()
+    ts = []
+    for _ in range(20):
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record()
+        vab.linear(x, w, b, out=y, workspace=ws)
+        e1.record()
+        e1.synchronize()
+        ts.append(e0.elapsed_time(e1) * 1e3)
+    us = statistics.median(ts)
+    peaks = measured_peaks()
+    print(json.dumps({"mode": "linear", "M": M, "K": K, "N": N, "us": us,
+                      "tflops": 2.0 * M * N * K / us / 1e6,
+                      "frac_bf16": 2.0 * M * N * K / us / 1e-6 / (peaks["bf16_tflops"] * 1e12),
+                      "peak_source": peaks["source"]}), flush=True)
+
+
 def main() -> None:
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -695,12 +737,17 @@ def main() -> None:
                     help="per-config report instead of the benchmark line (1 GPU)")
     ap.add_argument("--block", action="store_true",
                     help="the layers around attention, whole encoder layers and encoders (1 GPU)")
+    ap.add_argument("--linear", default=None, metavar="M,K,N",
+                    help="time one linear layer y = x w^T + bias of this shape (1 GPU)")
     args = ap.parse_args()
     if args.configs:
         run_configs(args)
         return
     if args.block:
         run_block(args)
+        return
+    if args.linear:
+        run_linear(args)
         return
 
     if "WORLD_SIZE" not in os.environ and args.gpus > 1:
