@@ -681,16 +681,20 @@ def run_block(args) -> None:
 
 
 def run_linear(args) -> None:
-    """One linear layer y = x w^T + bias on an (M, K, N) shape, seeded bf16 operands: five
-    warm calls, then the median of 20 CUDA-event timed calls (one JSON line).  Small enough
-    to run under ncu (the GEMM's profile)."""
+    """One linear layer y = x w^T + bias (+ a residual, or GELU) on an (M, K, N) shape with
+    seeded bf16 operands: five warm calls, then the median of 20 CUDA-event timed calls
+    (one JSON line).  Small enough to run under ncu (the GEMM's profile)."""
     import math as _m
 
     import torch
 
     import vit_self_attention_b200 as vab
 
-    M, K, N = (int(v) for v in args.linear.split(","))
+    fields = args.linear.split(",")
+    M, K, N = (int(v) for v in fields[:3])
+    epi = fields[3] if len(fields) > 3 else "bias"
+    if epi not in ("bias", "res", "gelu"):
+        raise SystemExit("--linear M,K,N[,bias|res|gelu]")
     dev = torch.device("cuda", 0)
     torch.cuda.set_device(dev)
 
@@ -700,22 +704,30 @@ def run_linear(args) -> None:
 
     x, w, b = t_((M, K), 1.0, 21), t_((N, K), 1.0 / _m.sqrt(K), 22), t_((N,), 0.1, 23)
     y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+    r = t_((M, N), 1.0, 24) if epi == "res" else None
     ws = torch.empty(vab.vla_linear_workspace_bytes(), dtype=torch.uint8, device=dev)
+
+    def call():
+        if epi == "gelu":
+            vab.linear_gelu(x, w, b, out=y, workspace=ws)
+        else:
+            vab.linear(x, w, b, res=r, out=y, workspace=ws)
+
     for _ in range(5):
-        vab.linear(x, w, b, out=y, workspace=ws)
+        call()
     torch.cuda.synchronize()
     ts = []
     for _ in range(20):
         e0 = torch.cuda.Event(enable_timing=True)
         e1 = torch.cuda.Event(enable_timing=True)
         e0.record()
-        vab.linear(x, w, b, out=y, workspace=ws)
+        call()
         e1.record()
         e1.synchronize()
         ts.append(e0.elapsed_time(e1) * 1e3)
     us = statistics.median(ts)
     peaks = measured_peaks()
-    print(json.dumps({"mode": "linear", "M": M, "K": K, "N": N, "us": us,
+    print(json.dumps({"mode": "linear", "M": M, "K": K, "N": N, "epilogue": epi, "us": us,
                       "tflops": 2.0 * M * N * K / us / 1e6,
                       "frac_bf16": 2.0 * M * N * K / us / 1e-6 / (peaks["bf16_tflops"] * 1e12),
                       "peak_source": peaks["source"]}), flush=True)
@@ -737,8 +749,9 @@ def main() -> None:
                     help="per-config report instead of the benchmark line (1 GPU)")
     ap.add_argument("--block", action="store_true",
                     help="the layers around attention, whole encoder layers and encoders (1 GPU)")
-    ap.add_argument("--linear", default=None, metavar="M,K,N",
-                    help="time one linear layer y = x w^T + bias of this shape (1 GPU)")
+    ap.add_argument("--linear", default=None, metavar="M,K,N[,bias|res|gelu]",
+                    help="time one linear layer y = x w^T + bias (+ residual, or GELU) of this "
+                         "shape (1 GPU)")
     args = ap.parse_args()
     if args.configs:
         run_configs(args)

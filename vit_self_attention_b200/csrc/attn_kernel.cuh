@@ -9,10 +9,11 @@
 // goes to memory; section 3.2: the qkv linear feeds the attention module).
 //
 // Blackwell mapping (one persistent CTA per SM, 384 threads = 3 warpgroups):
-//   warp 1      TMA producer: Q tiles (128 query rows) into two Q slots, K and
-//               V blocks (BK keys) into a ring of `ring` slots.  With `reuse`,
-//               a head's K/V blocks are loaded once and serve all of that
-//               head's Q tiles.
+//   warp 1      TMA producer: Q tiles (128 query rows) into one or two
+//               buffers per Q slot (with two, the next round's tile loads
+//               while the current round runs), K and V blocks (BK keys) into
+//               a ring of `ring` slots.  With `reuse`, a head's K/V blocks are
+//               loaded once and serve all of that head's Q tiles.
 //   warp 0      tcgen05 issuer of S = Q K^T into tensor memory (SS MMA, M=128,
 //               N=keys of the block, K=16 steps over d).
 //   warp 2      tcgen05 issuer of O += P V with P read from tensor memory (TS
@@ -21,8 +22,9 @@
 //               (= tensor-memory lane): online softmax in fp32 with exp2 and a
 //               pre-scaled log2(e), P as bf16 pairs in its own tensor-memory
 //               columns, O rescaled in tensor memory only when the running
-//               maximum grows by more than 2^8, epilogue O / l -> bf16 with
-//               16-byte stores.
+//               maximum grows by more than 2^8, epilogue O / l -> bf16 into
+//               a per-warp shared-memory buffer written out by one TMA store
+//               of the warp's 32 rows (whole 128-byte rows per transaction).
 //   warp 3      idle.
 //
 // Schedule.  A round holds up to two 128-row Q tiles, one per Q slot and
@@ -47,10 +49,11 @@
 // +BK+DP (BK/2 columns of bf16 pairs).  d=64 uses BK=128 (128+64+64 = 256),
 // d=72 uses BK=112 (112+80+56 = 248).
 //
-// Shared memory: a tile row holds channels 0..63 in a 128-byte-swizzled
-// region (TMA box {64,1,1,rows,1}); for d=72 channels 64..79 (72..79
-// zero-filled by TMA) sit in a 32-byte-swizzled region.  Q and K are read
-// K-major by the MMA, V MN-major.
+// Shared memory: Q buffers, the K/V ring, the output staging (8 warps x 32
+// rows, 128-byte swizzled), barriers.  A tile row holds channels 0..63 in a
+// 128-byte-swizzled region (TMA box {64,1,1,rows,1}); for d=72 channels
+// 64..79 (72..79 zero-filled by TMA) sit in a 32-byte-swizzled region.  Q and
+// K are read K-major by the MMA, V MN-major.
 //
 // Every mbarrier wait is bounded; a wait that runs out sets a shared abort
 // flag and the device status word, every role then leaves its loop, the
@@ -76,7 +79,8 @@ constexpr int kSoftmaxWarp0 = 4;
 constexpr int kThreads = 384;
 constexpr int kMaxRing = 6;
 constexpr uint32_t kTmemCols = 512;
-constexpr int kNumBarriers = 12 + 4 * kMaxRing + 3;
+constexpr int kMaxQBuf = 2;  // Q buffers per slot
+constexpr int kNumBarriers = 16 + 4 * kMaxRing + 3;
 constexpr uint32_t kBarrierRegionBytes = 512;  // barriers + tmem address + abort flag
 constexpr uint32_t kAlignSlack = 1024;
 constexpr unsigned long long kDrainLimitNs = 100000000ull;
@@ -125,6 +129,11 @@ struct Geom {
   static constexpr uint32_t kKVTail = BK * 128;
   static constexpr uint32_t kKVBytes = kKVTail + (kHasTail ? BK * 32 : 0);
   static constexpr uint32_t kKVStride = (kKVBytes + 1023u) & ~1023u;
+  // Output staging: per softmax warp 32 rows x 128 B (128-byte swizzled)
+  // [+ 32 rows x 16 B for channels 64..71 of d=72], written by TMA stores.
+  static constexpr uint32_t kStageWarp = 32 * 128;
+  static constexpr uint32_t kStageTailWarp = 32 * 16;
+  static constexpr uint32_t kStageBytes = 8 * kStageWarp + (kHasTail ? 8 * kStageTailWarp : 0);
   // Tensor-memory columns within a slot.
   static constexpr uint32_t kColO = BK;
   static constexpr uint32_t kColP = BK + DP;
@@ -136,7 +145,8 @@ struct AttnParams {
   CUtensorMap tm_q_tail;   // 32B-swizzled box {16, 1, 1, 128, 1}, channels 64..79 (d = 72)
   CUtensorMap tm_kv;       // 128B-swizzled box {64, 1, 1, BK, 1} (K / V blocks)
   CUtensorMap tm_kv_tail;  // 32B-swizzled box {16, 1, 1, BK, 1} (d = 72)
-  __nv_bfloat16* o;        // [B, N, H, d]
+  CUtensorMap tm_o;        // O as [B, N, H, d]: 128B-swizzled box {64, 1, 32, 1}
+  CUtensorMap tm_o_tail;   // unswizzled box {8, 1, 32, 1} at channel 64 (d = 72)
   int B, N, H;
   int num_kblocks;         // ceil(N / BK)
   int num_qtiles;          // ceil(N / 128)
@@ -153,29 +163,33 @@ struct AttnParams {
   int test_stall;          // testing hook: softmax warps wait on a barrier nothing completes
   int stream;              // 1: a CTA pairs its heads' Q tiles across head boundaries
                            // (whole heads with an odd tile count), K/V streamed
+  int qbuf;                // Q buffers per slot (1 or 2): with 2 the next round's Q tile
+                           // loads while the current round runs
 };
 
 template <int D>
-__host__ __device__ constexpr uint32_t smem_bytes_for_ring(int ring) {
-  return 2u * Geom<D>::kQBytes + 2u * static_cast<uint32_t>(ring) * Geom<D>::kKVStride +
+__host__ __device__ constexpr uint32_t smem_bytes_for(int ring, int qbuf) {
+  return 2u * static_cast<uint32_t>(qbuf) * Geom<D>::kQBytes +
+         2u * static_cast<uint32_t>(ring) * Geom<D>::kKVStride + Geom<D>::kStageBytes +
          kBarrierRegionBytes + kAlignSlack;
 }
 
 struct Barriers {
   uint32_t base;
-  __device__ uint32_t q_full(int s) const { return base + 8u * (0 + s); }
-  __device__ uint32_t q_empty(int s) const { return base + 8u * (2 + s); }
-  __device__ uint32_t s_full(int s) const { return base + 8u * (4 + s); }   // S in TMEM
-  __device__ uint32_t s_free(int s) const { return base + 8u * (6 + s); }   // S read out
-  __device__ uint32_t p_full(int s) const { return base + 8u * (8 + s); }   // P in TMEM
-  __device__ uint32_t o_prog(int s) const { return base + 8u * (10 + s); }  // each P V done
-  __device__ uint32_t k_full(int i) const { return base + 8u * (12 + i); }
-  __device__ uint32_t k_empty(int i) const { return base + 8u * (12 + kMaxRing + i); }
-  __device__ uint32_t v_full(int i) const { return base + 8u * (12 + 2 * kMaxRing + i); }
-  __device__ uint32_t v_empty(int i) const { return base + 8u * (12 + 3 * kMaxRing + i); }
-  __device__ uint32_t drain(int i) const { return base + 8u * (12 + 4 * kMaxRing + i); }
+  // Q buffer i = slot * qbuf + (the slot's Q load count mod qbuf).
+  __device__ uint32_t q_full(int i) const { return base + 8u * (0 + i); }
+  __device__ uint32_t q_empty(int i) const { return base + 8u * (4 + i); }
+  __device__ uint32_t s_full(int s) const { return base + 8u * (8 + s); }   // S in TMEM
+  __device__ uint32_t s_free(int s) const { return base + 8u * (10 + s); }  // S read out
+  __device__ uint32_t p_full(int s) const { return base + 8u * (12 + s); }  // P in TMEM
+  __device__ uint32_t o_prog(int s) const { return base + 8u * (14 + s); }  // each P V done
+  __device__ uint32_t k_full(int i) const { return base + 8u * (16 + i); }
+  __device__ uint32_t k_empty(int i) const { return base + 8u * (16 + kMaxRing + i); }
+  __device__ uint32_t v_full(int i) const { return base + 8u * (16 + 2 * kMaxRing + i); }
+  __device__ uint32_t v_empty(int i) const { return base + 8u * (16 + 3 * kMaxRing + i); }
+  __device__ uint32_t drain(int i) const { return base + 8u * (16 + 4 * kMaxRing + i); }
   // Never arrived at: the testing hook's wait runs out on it.
-  __device__ uint32_t never() const { return base + 8u * (12 + 4 * kMaxRing + 2); }
+  __device__ uint32_t never() const { return base + 8u * (16 + 4 * kMaxRing + 2); }
 };
 
 // Bounded wait for the phase of `bar` with the given parity, executed by a
@@ -334,7 +348,7 @@ __device__ void load_role(const AttnParams& p, uint32_t sQ, uint32_t sK, uint32_
   using G = Geom<D>;
   const int R = p.ring;
   const int nb = p.num_kblocks;
-  uint32_t nq0 = 0, nq1 = 0;  // Q loads issued into slot 0 / 1
+  uint32_t nq0 = 0, nq1 = 0;  // Q loads issued for slot 0 / 1
   uint32_t kv_ev = 0;         // K/V load events issued
   RingPos pos{0, 0u};         // ring position of the next K/V event
   bool ok = true;
@@ -342,15 +356,18 @@ __device__ void load_role(const AttnParams& p, uint32_t sQ, uint32_t sK, uint32_
   // The whole warp runs this loop and waits together; one lane issues.
   auto load_q = [&](int s, const Round& x) -> bool {
     const uint32_t nq = s == 0 ? nq0 : nq1;
-    if (!wait_bounded(bar.q_empty(s), (nq & 1u) ^ 1u, abort_flag, p.wait_limit_ns, kSiteLoadQ))
+    const uint32_t qb = static_cast<uint32_t>(p.qbuf);
+    const int qi = s * p.qbuf + static_cast<int>(nq % qb);  // Q buffer of this load
+    if (!wait_bounded(bar.q_empty(qi), ((nq / qb) & 1u) ^ 1u, abort_flag, p.wait_limit_ns,
+                      kSiteLoadQ))
       return false;
     if (elect_one()) {
-      const uint32_t dst = sQ + s * G::kQBytes;
+      const uint32_t dst = sQ + qi * G::kQBytes;
       const int row0 = x.tile(s) * kQRows;
-      mbar_arrive_expect_tx(bar.q_full(s), G::kQBytes);
-      tma_load_5d(dst, &p.tm_q, bar.q_full(s), 0, x.h(s), 0, row0, x.b(s));
+      mbar_arrive_expect_tx(bar.q_full(qi), G::kQBytes);
+      tma_load_5d(dst, &p.tm_q, bar.q_full(qi), 0, x.h(s), 0, row0, x.b(s));
       if (G::kHasTail)
-        tma_load_5d(dst + G::kQTail, &p.tm_q_tail, bar.q_full(s), 64, x.h(s), 0, row0, x.b(s));
+        tma_load_5d(dst + G::kQTail, &p.tm_q_tail, bar.q_full(qi), 64, x.h(s), 0, row0, x.b(s));
     }
     __syncwarp();
     if (s == 0) ++nq0; else ++nq1;
@@ -399,8 +416,13 @@ __device__ void load_role(const AttnParams& p, uint32_t sQ, uint32_t sK, uint32_
     }
   }
   // Wait (bounded) until every copy this thread issued has landed.
-  if (nq0 > 0) wait_drain(bar.q_full(0), (nq0 - 1u) & 1u, kDrainLimitNs);
-  if (nq1 > 0) wait_drain(bar.q_full(1), (nq1 - 1u) & 1u, kDrainLimitNs);
+  for (int s = 0; s < 2; ++s) {
+    for (int k = 0; k < p.qbuf; ++k) {
+      const uint32_t loads = ((s == 0 ? nq0 : nq1) + static_cast<uint32_t>(p.qbuf - 1 - k)) /
+                             static_cast<uint32_t>(p.qbuf);  // loads into buffer s * qbuf + k
+      if (loads > 0) wait_drain(bar.q_full(s * p.qbuf + k), (loads - 1u) & 1u, kDrainLimitNs);
+    }
+  }
   for (int i = 0; i < R; ++i) {
     const uint32_t arms = kv_ev / R + (static_cast<uint32_t>(i) < kv_ev % R ? 1u : 0u);
     if (arms > 0) {
@@ -426,7 +448,8 @@ __device__ void mma_role(const AttnParams& p, uint32_t tmem, uint32_t sQ, uint32
   const int R = p.ring;
   const int nb = p.num_kblocks;
   const unsigned long long lim = p.wait_limit_ns;
-  uint32_t nq0 = 0, nq1 = 0;  // q_full phases consumed per Q slot
+  uint32_t nq0 = 0, nq1 = 0;  // Q tiles consumed per slot
+  int qi0 = 0, qi1 = 0;       // Q buffer of the current round per slot
   uint32_t nf0 = 0, nf1 = 0;  // s_free phases consumed per slot
   uint32_t np0 = 0, np1 = 0;  // p_full phases consumed per slot
   RingPos pos{0, 0u};         // ring position of the next unit / round's first K/V event
@@ -437,7 +460,7 @@ __device__ void mma_role(const AttnParams& p, uint32_t tmem, uint32_t sQ, uint32
   const uint64_t k_tail0 = smem_desc(sK + G::kKVTail, 16, 256, kSwizzle32);
   const uint64_t v_desc0 = smem_desc(sV, G::kKVTail, 1024, kSwizzle128);
   const uint64_t v_tail0 = smem_desc(sV + G::kKVTail, 32 * G::BK, 256, kSwizzle32);
-  constexpr uint64_t kQStep = G::kQBytes >> 4;     // next Q slot
+  constexpr uint64_t kQStep = G::kQBytes >> 4;     // next Q buffer
   constexpr uint64_t kKVStep = G::kKVStride >> 4;  // next ring slot
   constexpr uint32_t kIdescPV = idesc_bf16_m128(64u, 1u);
   constexpr uint32_t kIdescPVTail = idesc_bf16_m128(16u, 1u);
@@ -455,8 +478,16 @@ __device__ void mma_role(const AttnParams& p, uint32_t tmem, uint32_t sQ, uint32
   };
   auto wait_q = [&](int s) -> bool {
     const uint32_t nq = s == 0 ? nq0 : nq1;
-    if (!wait_bounded(bar.q_full(s), nq & 1u, abort_flag, lim, kSiteMmaQ)) return false;
-    if (s == 0) ++nq0; else ++nq1;
+    const uint32_t qb = static_cast<uint32_t>(p.qbuf);
+    const int qi = s * p.qbuf + static_cast<int>(nq % qb);
+    if (!wait_bounded(bar.q_full(qi), (nq / qb) & 1u, abort_flag, lim, kSiteMmaQ)) return false;
+    if (s == 0) {
+      ++nq0;
+      qi0 = qi;
+    } else {
+      ++nq1;
+      qi1 = qi;
+    }
     tc_fence_after();
     return true;
   };
@@ -487,14 +518,15 @@ __device__ void mma_role(const AttnParams& p, uint32_t tmem, uint32_t sQ, uint32
     VLA_TRACE_EVENT(kTrMmaS, s, j);
     const uint32_t idesc = idesc_bf16_m128(static_cast<uint32_t>(block_cols<G::BK>(p.N, j)), 0u);
     const uint32_t d_tmem = tmem + s * 256;
-    const uint64_t qd = q_desc0 + s * kQStep;
+    const int qi = s == 0 ? qi0 : qi1;
+    const uint64_t qd = q_desc0 + qi * kQStep;
     const uint64_t kd = k_desc0 + kslot * kKVStep;
     if (elect_one()) {
 #pragma unroll
       for (int kk = 0; kk < 4; ++kk)
         mma_ss(d_tmem, qd + 2 * kk, kd + 2 * kk, idesc, kk > 0 ? 1u : 0u);  // 16 ch = 32 B
       if (G::kHasTail)
-        mma_ss(d_tmem, q_tail0 + s * kQStep, k_tail0 + kslot * kKVStep, idesc, 1u);
+        mma_ss(d_tmem, q_tail0 + qi * kQStep, k_tail0 + kslot * kKVStep, idesc, 1u);
       mma_commit(bar.s_full(s));
     }
     __syncwarp();
@@ -536,7 +568,7 @@ __device__ void mma_role(const AttnParams& p, uint32_t tmem, uint32_t sQ, uint32
           if ((!sh || s == 0) && !(ok = wait_k(cur))) break;
           if (!(ok = (j == 0 ? wait_q(s) : wait_free(s)))) break;
           scores(s, j, cur.slot);
-          if (j == nb - 1) commit(bar.q_empty(s));
+          if (j == nb - 1) commit(bar.q_empty(s == 0 ? qi0 : qi1));
           if (!sh) {
             if (release) commit(bar.k_empty(cur.slot));
             cur.advance(R);
@@ -593,14 +625,12 @@ constexpr int kPolyEvery = 16;
 
 // One key block for one query row.  Reads S (NC columns at compile time,
 // nvalid valid at run time), signals that S has been read, updates the
-// running max / sum, stores P, rescales O when the maximum grew.  Returns
-// false on abort.
+// running max / sum and leaves P (bf16 pairs, zero past NC) in pk.  Returns
+// whether the warp must rescale O by alpha (warp-uniform).
 template <int D, int NC>
 __device__ __forceinline__ bool softmax_block(const AttnParams& p, SoftState& st, uint32_t tS,
-                                              uint32_t tO, uint32_t tP, int nvalid, int j,
-                                              const Barriers& bar, int s, uint32_t o_parity,
-                                              volatile int* abort_flag, int lane) {
-  using G = Geom<D>;
+                                              int nvalid, int j, const Barriers& bar, int s,
+                                              int lane, uint32_t (&pk)[64], float& alpha) {
   const float c = p.c;
   float x[NC];
   {
@@ -638,7 +668,7 @@ __device__ __forceinline__ bool softmax_block(const AttnParams& p, SoftState& st
   // stay below 2^8.
   const bool grow = (m_blk - st.m_run) * c > 8.0f;
   const bool rescale = __any_sync(0xffffffffu, grow);
-  float alpha = 1.0f;
+  alpha = 1.0f;
   if (rescale) {
     const float m_new = fmaxf(st.m_run, m_blk);
     alpha = ex2_approx((st.m_run - m_new) * c);
@@ -651,7 +681,6 @@ __device__ __forceinline__ bool softmax_block(const AttnParams& p, SoftState& st
   const uint64_t c2 = f32x2_pack(c, c);
   const uint64_t nmc2 = f32x2_pack(-mc, -mc);
   uint64_t acc2[2] = {0ull, 0ull};
-  uint32_t pk[64];
 #pragma unroll
   for (int i = 0; i < NC / 2; ++i) {
     const uint64_t a = f32x2_fma(f32x2_pack(x[2 * i], x[2 * i + 1]), c2, nmc2);
@@ -674,40 +703,15 @@ __device__ __forceinline__ bool softmax_block(const AttnParams& p, SoftState& st
   for (int i = NC / 2; i < 64; ++i) pk[i] = 0u;
   VLA_TRACE_EVENT(kTrSoftExp, s, j);
   st.l_run += (lsum[0] + lsum[1]) + (lsum[2] + lsum[3]);
-  if (j > 0) {
-    // P V of the previous block must be done before P is overwritten and
-    // before O is touched (this observes every phase of o_prog in order).
-    if (!wait_bounded(bar.o_prog(s), o_parity, abort_flag, p.wait_limit_ns, kSiteSoftO))
-      return false;
-    tc_fence_after();
-  }
-  tmem_st64(tP, pk);
-  if (j > 0 && rescale) {
-    uint32_t ob[64];
-    tmem_ld64(tO, ob);
-#pragma unroll
-    for (int i = 0; i < 64; ++i) ob[i] = __float_as_uint(__uint_as_float(ob[i]) * alpha);
-    tmem_st64(tO, ob);
-    if (G::DP > 64) {
-      uint32_t ot[16];
-      tmem_ld16(tO + 64, ot);
-#pragma unroll
-      for (int i = 0; i < 16; ++i) ot[i] = __float_as_uint(__uint_as_float(ot[i]) * alpha);
-      tmem_st16(tO + 64, ot);
-    }
-  }
-  tmem_wait_st();
-  return true;
+  return rescale;
 }
 
 template <int D>
 __device__ __forceinline__ bool softmax_block_dispatch(const AttnParams& p, SoftState& st,
-                                                       uint32_t tS, uint32_t tO, uint32_t tP,
-                                                       int ncols, int nvalid, int j,
-                                                       const Barriers& bar, int s, uint32_t op,
-                                                       volatile int* abort_flag, int lane) {
-#define VLA_SB(NC) \
-  return softmax_block<D, NC>(p, st, tS, tO, tP, nvalid, j, bar, s, op, abort_flag, lane)
+                                                       uint32_t tS, int ncols, int nvalid, int j,
+                                                       const Barriers& bar, int s, int lane,
+                                                       uint32_t (&pk)[64], float& alpha) {
+#define VLA_SB(NC) return softmax_block<D, NC>(p, st, tS, nvalid, j, bar, s, lane, pk, alpha)
   if (ncols >= Geom<D>::BK) VLA_SB(Geom<D>::BK);
   switch (ncols) {
     case 112: VLA_SB(112);
@@ -721,32 +725,91 @@ __device__ __forceinline__ bool softmax_block_dispatch(const AttnParams& p, Soft
 #undef VLA_SB
 }
 
+// Where a finished round's output goes: image, head and first row of this
+// warp's 32 rows, and 1 / l for this thread's row.
+struct OutRow {
+  int b, h, row0;
+  float inv_l;
+};
+
+// O / l -> bf16 for this warp's 32 rows through its shared-memory staging
+// buffer (128-byte swizzle: 16-byte chunk t of row r at chunk t ^ (r mod 8),
+// so the eight rows of a store phase hit distinct banks), then one TMA
+// store of the 32 x d box; rows past N fall outside the tensor and are not
+// written.  The tensor-memory loads are warp-collective.
 template <int D>
-__device__ void softmax_role(const AttnParams& p, uint32_t tmem, const Barriers& bar,
-                             volatile int* abort_flag, int warp, int lane) {
+__device__ __forceinline__ void store_output(const AttnParams& p, uint32_t tO, const OutRow& r,
+                                             uint32_t stage, uint32_t stage_tail, int lane) {
+  using G = Geom<D>;
+  uint32_t ob[64];
+  tmem_ld64(tO, ob);
+  uint32_t ot[16];
+  if (G::DP > 64) tmem_ld16(tO + 64, ot);
+  if (r.row0 >= p.N) return;  // warp-uniform: no row of this warp is a token
+  // The previous store from this buffer must have finished reading it.
+  if (lane == 0) bulk_wait_read<0>();
+  __syncwarp();
+  const uint32_t row_s = stage + static_cast<uint32_t>(lane) * 128u;
+#pragma unroll
+  for (int t = 0; t < 8; ++t) {
+    float v[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) v[e] = __uint_as_float(ob[8 * t + e]) * r.inv_l;
+    st_shared_v4(row_s + ((static_cast<uint32_t>(t) ^ (lane & 7u)) << 4), pack_bf16x2(v[0], v[1]),
+                 pack_bf16x2(v[2], v[3]), pack_bf16x2(v[4], v[5]), pack_bf16x2(v[6], v[7]));
+  }
+  if (G::kHasTail) {
+    float v[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) v[e] = __uint_as_float(ot[e]) * r.inv_l;
+    st_shared_v4(stage_tail + static_cast<uint32_t>(lane) * 16u, pack_bf16x2(v[0], v[1]),
+                 pack_bf16x2(v[2], v[3]), pack_bf16x2(v[4], v[5]), pack_bf16x2(v[6], v[7]));
+  }
+  fence_async_shared();
+  __syncwarp();
+  if (lane == 0) {
+    tma_store_4d(&p.tm_o, stage, 0, r.h, r.row0, r.b);
+    if (G::kHasTail) tma_store_4d(&p.tm_o_tail, stage_tail, 64, r.h, r.row0, r.b);
+    bulk_commit();
+  }
+}
+
+// Softmax warpgroup of Q slot s.  Per key block: read S, exponentials, then
+// (after the previous P V has finished with the P columns) store P; after a
+// round's last block, O / l of its Q tile to the output.
+
+template <int D>
+__device__ void softmax_loop(const AttnParams& p, uint32_t tmem, const Barriers& bar,
+                             volatile int* abort_flag, int warp, int lane, uint32_t stage,
+                             uint32_t stage_tail) {
   using G = Geom<D>;
   const int s = (warp - kSoftmaxWarp0) >> 2;  // Q slot of this warpgroup
   const int quad = warp & 3;
-  const int row_in_tile = quad * 32 + lane;
   const uint32_t lane_bits = static_cast<uint32_t>(quad * 32) << 16;
   const uint32_t tS = tmem + lane_bits + s * 256;
   const uint32_t tO = tS + G::kColO;
   const uint32_t tP = tS + G::kColP;
   const int nb = p.num_kblocks;
   uint32_t ns = 0;   // s_full phases consumed
-  uint32_t npv = 0;  // o_prog phases consumed
+  uint32_t nop = 0;  // o_prog phases consumed
   if (p.test_stall) {
     // Testing hook: a wait that nothing completes runs out after the bound,
     // which takes the whole CTA down the error path.
     (void)wait_bounded(bar.never(), 0u, abort_flag, p.wait_limit_ns, kSiteTestStall);
     return;
   }
+  auto wait_pv = [&]() -> bool {
+    if (!wait_bounded(bar.o_prog(s), nop & 1u, abort_flag, p.wait_limit_ns, kSiteSoftO))
+      return false;
+    ++nop;
+    tc_fence_after();
+    return true;
+  };
 
   for (Cursor cu = cursor_start(); cursor_more(p, cu);) {
     const Round x = next_round(p, cu);
     const bool full = x.nslots == 2;
     if (!full && s == 1) continue;
-    const int tile = x.tile(s);
     SoftState st{-INFINITY, 0.0f};
     for (int j = 0; j < nb; ++j) {
       if (!wait_bounded(bar.s_full(s), ns & 1u, abort_flag, p.wait_limit_ns, kSiteSoftS))
@@ -754,48 +817,54 @@ __device__ void softmax_role(const AttnParams& p, uint32_t tmem, const Barriers&
       ++ns;
       tc_fence_after();
       VLA_TRACE_EVENT(kTrSoftS, s, j);
-      const bool ok = softmax_block_dispatch<D>(
-          p, st, tS, tO, tP, block_cols<G::BK>(p.N, j), min(G::BK, p.N - j * G::BK), j, bar, s,
-          (npv + j - 1) & 1u, abort_flag, lane);
-      if (!ok) return;
+      uint32_t pk[64];
+      float alpha;
+      const bool rescale = softmax_block_dispatch<D>(p, st, tS, block_cols<G::BK>(p.N, j),
+                                                     min(G::BK, p.N - j * G::BK), j, bar, s,
+                                                     lane, pk, alpha);
+      // P V of the previous block must be done before P is overwritten and
+      // before O is touched (this observes every phase of o_prog in order).
+      if (j > 0) {
+        if (!wait_pv()) return;
+      }
+      tmem_st64(tP, pk);
+      if (j > 0 && rescale) {
+        uint32_t ob[64];
+        tmem_ld64(tO, ob);
+#pragma unroll
+        for (int i = 0; i < 64; ++i) ob[i] = __float_as_uint(__uint_as_float(ob[i]) * alpha);
+        tmem_st64(tO, ob);
+        if (G::DP > 64) {
+          uint32_t ot[16];
+          tmem_ld16(tO + 64, ot);
+#pragma unroll
+          for (int i = 0; i < 16; ++i) ot[i] = __float_as_uint(__uint_as_float(ot[i]) * alpha);
+          tmem_st16(tO + 64, ot);
+        }
+      }
+      tmem_wait_st();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(bar.p_full(s));
       VLA_TRACE_EVENT(kTrSoftP, s, j);
     }
-    // Epilogue: wait for the last P V, then O / l -> bf16, 16-byte stores.
-    if (!wait_bounded(bar.o_prog(s), (npv + nb - 1) & 1u, abort_flag, p.wait_limit_ns,
-                      kSiteSoftO))
-      return;
-    npv += nb;
-    tc_fence_after();
+    // Epilogue: the last P V, then O / l.
+    if (!wait_pv()) return;
     VLA_TRACE_EVENT(kTrSoftEpi, s, 0);
-    const float inv_l = 1.0f / st.l_run;
-    uint32_t ob[64];
-    tmem_ld64(tO, ob);
-    uint32_t ot[16];
-    if (G::DP > 64) tmem_ld16(tO + 64, ot);
-    const int row = tile * kQRows + row_in_tile;
-    if (row < p.N) {
-      uint4* dst = reinterpret_cast<uint4*>(
-          p.o + ((static_cast<size_t>(x.b(s)) * p.N + row) * p.H + x.h(s)) * D);
-#pragma unroll
-      for (int t = 0; t < D / 8; ++t) {
-        float v[8];
-#pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          const int ch = 8 * t + e;
-          v[e] = __uint_as_float(ch < 64 ? ob[ch] : ot[ch - 64]) * inv_l;
-        }
-        uint4 w;
-        w.x = pack_bf16x2(v[0], v[1]);
-        w.y = pack_bf16x2(v[2], v[3]);
-        w.z = pack_bf16x2(v[4], v[5]);
-        w.w = pack_bf16x2(v[6], v[7]);
-        dst[t] = w;
-      }
-    }
+    const OutRow r{x.b(s), x.h(s), x.tile(s) * kQRows + quad * 32, 1.0f / st.l_run};
+    store_output<D>(p, tO, r, stage, stage_tail, lane);
   }
+}
+
+template <int D>
+__device__ void softmax_role(const AttnParams& p, uint32_t tmem, const Barriers& bar,
+                             volatile int* abort_flag, int warp, int lane, uint32_t stage,
+                             uint32_t stage_tail) {
+  softmax_loop<D>(p, tmem, bar, abort_flag, warp, lane, stage, stage_tail);
+  // This warp's output stores must have read the staging buffer (and
+  // completed) before the CTA ends, on every path out of the loop.
+  if (lane == 0) bulk_wait_all();
+  __syncwarp();
 }
 
 // ------------------------------------------------------------ kernel
@@ -806,9 +875,10 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
   const uint32_t sQ = base;
-  const uint32_t sK = sQ + 2 * G::kQBytes;
+  const uint32_t sK = sQ + 2 * p.qbuf * G::kQBytes;
   const uint32_t sV = sK + p.ring * G::kKVStride;
-  const uint32_t sBar = sV + p.ring * G::kKVStride;
+  const uint32_t sStage = sV + p.ring * G::kKVStride;
+  const uint32_t sBar = sStage + G::kStageBytes;
   uint8_t* bar_generic = smem_raw + (sBar - raw);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_generic + 8 * kNumBarriers);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(bar_generic + 8 * kNumBarriers + 4);
@@ -818,9 +888,11 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
   const int lane = threadIdx.x & 31;
 
   if (threadIdx.x == 0) {
+    for (int i = 0; i < 2 * kMaxQBuf; ++i) {
+      mbar_init(bar.q_full(i), 1);
+      mbar_init(bar.q_empty(i), 1);
+    }
     for (int s = 0; s < 2; ++s) {
-      mbar_init(bar.q_full(s), 1);
-      mbar_init(bar.q_empty(s), 1);
       mbar_init(bar.s_full(s), 1);
       mbar_init(bar.s_free(s), 4);
       mbar_init(bar.p_full(s), 4);
@@ -842,9 +914,11 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
   if (warp == kLoadWarp && lane == 0) {
     prefetch_tmap(&p.tm_q);
     prefetch_tmap(&p.tm_kv);
+    prefetch_tmap(&p.tm_o);
     if (G::kHasTail) {
       prefetch_tmap(&p.tm_q_tail);
       prefetch_tmap(&p.tm_kv_tail);
+      prefetch_tmap(&p.tm_o_tail);
     }
   }
   if (warp == kMmaWarp) {
@@ -867,7 +941,9 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
     mma_role<D>(p, tmem, sQ, sK, sV, bar, abort_flag, warp == kMmaWarp);
     __syncwarp();
   } else if (warp >= kSoftmaxWarp0) {
-    softmax_role<D>(p, tmem, bar, abort_flag, warp, lane);
+    const int ws = warp - kSoftmaxWarp0;  // staging buffer of this warp
+    softmax_role<D>(p, tmem, bar, abort_flag, warp, lane, sStage + ws * G::kStageWarp,
+                    sStage + 8 * G::kStageWarp + ws * G::kStageTailWarp);
     __syncwarp();
   }
 

@@ -121,28 +121,12 @@ struct GemmBarriers {
   }
 };
 
-// Tiled 2-D store of a shared-memory box to global memory (bulk group), and
-// the waits on this thread's bulk groups: until at most N of them still read
-// shared memory, and until all have completed.
+// Tiled 2-D store of a shared-memory box to global memory (bulk group).
 __device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, uint32_t src, int c0, int c1) {
   asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%1, %2}], [%3];" ::"l"(
                    reinterpret_cast<uint64_t>(map)),
                "r"(c0), "r"(c1), "r"(src)
                : "memory");
-}
-__device__ __forceinline__ void bulk_commit() {
-  asm volatile("cp.async.bulk.commit_group;" ::: "memory");
-}
-template <int N>
-__device__ __forceinline__ void bulk_wait_read() {
-  asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(N) : "memory");
-}
-__device__ __forceinline__ void bulk_wait_all() {
-  asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
-}
-// Makes this thread's shared-memory writes visible to the TMA unit.
-__device__ __forceinline__ void fence_async_shared() {
-  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
 // 2-D tiled load of one box into shared memory, completing on `bar`.
@@ -352,20 +336,42 @@ __device__ __forceinline__ uint4 epi8(const GemmParams& p, const uint32_t* acc, 
   return o;
 }
 
+// Epilogue state of one warp: staged chunks so far (they alternate between the
+// warp's two staging buffers) and the residual loads issued into them.
+struct EpiChunks {
+  uint32_t done = 0;       // chunks staged and stored
+  uint32_t res_issued = 0; // residual loads issued (chunk g's load is the g-th)
+};
+
 template <int BN>
-__device__ __forceinline__ void gemm_epilogue_role(const GemmParams& p, uint32_t tmem,
+__device__ __forceinline__ void gemm_epilogue_loop(const GemmParams& p, uint32_t tmem,
                                                    const GemmBarriers& bar,
                                                    volatile int* abort_flag, int warp, int lane,
-                                                   uint32_t staging) {
+                                                   uint32_t stg, EpiChunks& ch) {
   const int quad = warp & 3;
   const int ew = warp - kEpiWarp0;  // epilogue warp 0..3
-  const uint32_t stg = staging + static_cast<uint32_t>(ew) * 2u * kStageOutBytes;
-  uint32_t chunks_done = 0;         // staged chunks of this warp (alternating buffers)
+  uint32_t& chunks_done = ch.done;
   const int r_in = quad * 32 + lane;
   const uint32_t lane_bits = static_cast<uint32_t>(quad * 32) << 16;
   const size_t tile_elems = static_cast<size_t>(kBM) * BN;
   const int tiles = p.tiles_m * p.tiles_n;
+  // The residual of chunk g goes into buffer g % 2 one chunk ahead of its use
+  // (across tile boundaries too): issued right after chunk g-1's store, once
+  // the store of chunk g-2 (the buffer's last user) has finished reading it.
+  const bool prefetch = p.res != nullptr && p.splits == 1;
+  auto issue_res = [&](int n0, int row0) {
+    const uint32_t g = ch.res_issued;
+    const uint32_t rb = bar.res_full(ew, static_cast<int>(g & 1u));
+    if (lane == 0) {
+      bulk_wait_read<1>();
+      mbar_arrive_expect_tx(rb, kStageOutBytes);
+      tma_load_2d(stg + (g & 1u) * kStageOutBytes, &p.tm_res, rb, n0, row0);
+    }
+    __syncwarp();
+    ++ch.res_issued;
+  };
   Work wk;
+  if (prefetch && work_at(p, 0, wk)) issue_res(wk.nt * BN, wk.mt * kBM + quad * 32);
   for (int i = 0; work_at(p, i, wk); ++i) {
     const int buf = i & 1;
     if (!wait_bounded(bar.acc_full(buf), (i >> 1) & 1, abort_flag, p.wait_limit_ns, kSiteEpi))
@@ -456,17 +462,15 @@ __device__ __forceinline__ void gemm_epilogue_role(const GemmParams& p, uint32_t
       const int bsel = static_cast<int>(chunks_done & 1u);
       const uint32_t buf_s = stg + static_cast<uint32_t>(bsel) * kStageOutBytes;
       const int n0 = n_base + 64 * c;
-      // The store that last read this buffer must be done reading it.
-      if (lane == 0) bulk_wait_read<1>();
-      __syncwarp();
-      if (p.res != nullptr) {
-        const uint32_t rb = bar.res_full(ew, bsel);
-        if (lane == 0) {
-          mbar_arrive_expect_tx(rb, kStageOutBytes);
-          tma_load_2d(buf_s, &p.tm_res, rb, n0, row0);
-        }
-        if (!wait_bounded(rb, (chunks_done >> 1) & 1u, abort_flag, p.wait_limit_ns, kSiteEpi))
+      if (prefetch) {
+        // This chunk's residual was issued one chunk ago.
+        if (!wait_bounded(bar.res_full(ew, bsel), (chunks_done >> 1) & 1u, abort_flag,
+                          p.wait_limit_ns, kSiteEpi))
           return;
+      } else {
+        // The store that last read this buffer must be done reading it.
+        if (lane == 0) bulk_wait_read<1>();
+        __syncwarp();
       }
       uint32_t a[64];
       tmem_ld32(t + 64 * c, reinterpret_cast<uint32_t(&)[32]>(a[0]));
@@ -493,13 +497,35 @@ __device__ __forceinline__ void gemm_epilogue_role(const GemmParams& p, uint32_t
         bulk_commit();
       }
       ++chunks_done;
+      if (prefetch) {
+        Work nx;
+        if (c + 1 < BN / 64) {
+          issue_res(n0 + 64, row0);
+        } else if (work_at(p, i + 1, nx)) {
+          issue_res(nx.nt * BN, nx.mt * kBM + quad * 32);
+        }
+      }
     }
     (void)row;
     tc_fence_before();
     __syncwarp();
     if (lane == 0) mbar_arrive(bar.acc_empty(buf));
   }
-  // Every TMA store of this warp must have finished before the CTA exits.
+}
+
+template <int BN>
+__device__ __forceinline__ void gemm_epilogue_role(const GemmParams& p, uint32_t tmem,
+                                                   const GemmBarriers& bar,
+                                                   volatile int* abort_flag, int warp, int lane,
+                                                   uint32_t staging) {
+  const int ew = warp - kEpiWarp0;
+  const uint32_t stg = staging + static_cast<uint32_t>(ew) * 2u * kStageOutBytes;
+  EpiChunks ch;
+  gemm_epilogue_loop<BN>(p, tmem, bar, abort_flag, warp, lane, stg, ch);
+  // On every way out: residual loads issued but not waited for must land, and
+  // every TMA store of this warp must have finished, before the CTA exits.
+  for (uint32_t g = ch.done; g < ch.res_issued; ++g)
+    wait_drain(bar.res_full(ew, static_cast<int>(g & 1u)), (g >> 1) & 1u, kDrainLimitNs);
   if (lane == 0) bulk_wait_all();
   __syncwarp();
 }

@@ -230,6 +230,24 @@ int encode_map(const DriverFns& fns, CUtensorMap* map, const void* qkv, int B, i
   return rc == CUDA_SUCCESS ? VLA_ATTN_OK : VLA_ATTN_ERR_CUDA;
 }
 
+// O as a 4-D tensor [B, N, H, d] (d innermost) for the kernel's output
+// stores: box {box_c, 1, 32, 1} (32 rows of one head) at a channel offset.
+int encode_out_map(const DriverFns& fns, CUtensorMap* map, const void* o, int B, int N, int H,
+                   int d, uint32_t box_c, CUtensorMapSwizzle swizzle) {
+  const cuuint64_t dims[4] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(H),
+                              static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(B)};
+  const cuuint64_t row = static_cast<cuuint64_t>(H) * d * 2ull;
+  const cuuint64_t strides[3] = {static_cast<cuuint64_t>(d) * 2ull, row,
+                                 row * static_cast<cuuint64_t>(N)};
+  const cuuint32_t box[4] = {box_c, 1u, 32u, 1u};
+  const cuuint32_t elem_strides[4] = {1u, 1u, 1u, 1u};
+  const CUresult rc = fns.encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(o),
+                                 dims, strides, box, elem_strides, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                                 swizzle, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+                                 CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return rc == CUDA_SUCCESS ? VLA_ATTN_OK : VLA_ATTN_ERR_CUDA;
+}
+
 int check_args(const void* q, const void* k, const void* v, const void* o, int B, int N, int H,
                int d, float scale) {
   if (q == nullptr || k == nullptr || v == nullptr || o == nullptr) return VLA_ATTN_ERR_NULL;
@@ -249,38 +267,45 @@ int check_args(const void* q, const void* k, const void* v, const void* o, int B
   return VLA_ATTN_OK;
 }
 
-// Tensor maps of recent calls, in static host memory: a direct-mapped table keyed by
-// everything the maps encode (base address, shape, head dimension).  A hit skips the
-// 2-4 encodings of a call; the maps hold no pointer other than the base, so a buffer
-// freed and reallocated at the same address with the same shape reuses valid maps.
+// Tensor maps of recent calls, in static host memory: direct-mapped tables keyed by
+// everything the maps encode (base address, shape, head dimension), one for the QKV
+// input and one for the output.  A hit skips the encodings of a call; the maps hold
+// no pointer other than the base, so a buffer freed and reallocated at the same
+// address with the same shape reuses valid maps.
 struct MapSet {
   bool valid = false;
   const void* base = nullptr;
   int B = 0, N = 0, H = 0, d = 0;
-  CUtensorMap q, kv, q_tail, kv_tail;
+  CUtensorMap m0, m1, m2, m3;  // QKV: q, kv, q_tail, kv_tail; output: o, o_tail
 };
 constexpr int kMapCacheSlots = 64;
 std::mutex g_map_mutex;
 MapSet g_map_cache[kMapCacheSlots];
+MapSet g_out_map_cache[kMapCacheSlots];
 
-template <int D>
-int tensor_maps(const DriverFns& fns, const void* q, int B, int N, int H, vla::AttnParams* prm) {
-  using G = vla::Geom<D>;
-  const uint64_t h = (reinterpret_cast<uintptr_t>(q) >> 4) * 0x9E3779B97F4A7C15ull ^
+MapSet& map_slot(MapSet* table, const void* base, int B, int N, int H, int D) {
+  const uint64_t h = (reinterpret_cast<uintptr_t>(base) >> 4) * 0x9E3779B97F4A7C15ull ^
                      (static_cast<uint64_t>(B) * 73856093ull) ^ (static_cast<uint64_t>(N) << 20) ^
                      (static_cast<uint64_t>(H) << 40) ^ static_cast<uint64_t>(D);
+  return table[(h >> 32) % kMapCacheSlots];
+}
+
+template <int D>
+int tensor_maps(const DriverFns& fns, const void* q, const void* o, int B, int N, int H,
+                vla::AttnParams* prm) {
+  using G = vla::Geom<D>;
   std::lock_guard<std::mutex> lock(g_map_mutex);
-  MapSet& e = g_map_cache[(h >> 32) % kMapCacheSlots];
+  MapSet& e = map_slot(g_map_cache, q, B, N, H, D);
   if (!(e.valid && e.base == q && e.B == B && e.N == N && e.H == H && e.d == D)) {
     e.valid = false;
-    int rc = encode_map(fns, &e.q, q, B, N, H, D, 64u, vla::kQRows, CU_TENSOR_MAP_SWIZZLE_128B);
+    int rc = encode_map(fns, &e.m0, q, B, N, H, D, 64u, vla::kQRows, CU_TENSOR_MAP_SWIZZLE_128B);
     if (rc != VLA_ATTN_OK) return rc;
-    rc = encode_map(fns, &e.kv, q, B, N, H, D, 64u, G::BK, CU_TENSOR_MAP_SWIZZLE_128B);
+    rc = encode_map(fns, &e.m1, q, B, N, H, D, 64u, G::BK, CU_TENSOR_MAP_SWIZZLE_128B);
     if (rc != VLA_ATTN_OK) return rc;
     if (G::kHasTail) {
-      rc = encode_map(fns, &e.q_tail, q, B, N, H, D, 16u, vla::kQRows, CU_TENSOR_MAP_SWIZZLE_32B);
+      rc = encode_map(fns, &e.m2, q, B, N, H, D, 16u, vla::kQRows, CU_TENSOR_MAP_SWIZZLE_32B);
       if (rc != VLA_ATTN_OK) return rc;
-      rc = encode_map(fns, &e.kv_tail, q, B, N, H, D, 16u, G::BK, CU_TENSOR_MAP_SWIZZLE_32B);
+      rc = encode_map(fns, &e.m3, q, B, N, H, D, 16u, G::BK, CU_TENSOR_MAP_SWIZZLE_32B);
       if (rc != VLA_ATTN_OK) return rc;
     }
     e.base = q;
@@ -290,11 +315,29 @@ int tensor_maps(const DriverFns& fns, const void* q, int B, int N, int H, vla::A
     e.d = D;
     e.valid = true;
   }
-  prm->tm_q = e.q;
-  prm->tm_kv = e.kv;
+  MapSet& f = map_slot(g_out_map_cache, o, B, N, H, D);
+  if (!(f.valid && f.base == o && f.B == B && f.N == N && f.H == H && f.d == D)) {
+    f.valid = false;
+    int rc = encode_out_map(fns, &f.m0, o, B, N, H, D, 64u, CU_TENSOR_MAP_SWIZZLE_128B);
+    if (rc != VLA_ATTN_OK) return rc;
+    if (G::kHasTail) {
+      rc = encode_out_map(fns, &f.m1, o, B, N, H, D, 8u, CU_TENSOR_MAP_SWIZZLE_NONE);
+      if (rc != VLA_ATTN_OK) return rc;
+    }
+    f.base = o;
+    f.B = B;
+    f.N = N;
+    f.H = H;
+    f.d = D;
+    f.valid = true;
+  }
+  prm->tm_q = e.m0;
+  prm->tm_kv = e.m1;
+  prm->tm_o = f.m0;
   if (G::kHasTail) {
-    prm->tm_q_tail = e.q_tail;
-    prm->tm_kv_tail = e.kv_tail;
+    prm->tm_q_tail = e.m2;
+    prm->tm_kv_tail = e.m3;
+    prm->tm_o_tail = f.m1;
   }
   return VLA_ATTN_OK;
 }
@@ -305,21 +348,32 @@ int launch(const void* q, void* o, int B, int N, int H, float scale, cudaStream_
   using G = vla::Geom<D>;
   vla::AttnParams prm;
   std::memset(&prm, 0, sizeof(prm));
-  int rc = tensor_maps<D>(fns, q, B, N, H, &prm);
+  int rc = tensor_maps<D>(fns, q, o, B, N, H, &prm);
   if (rc != VLA_ATTN_OK) return rc;
   const int nb = (N + G::BK - 1) / G::BK;
   const int nq = (N + vla::kQRows - 1) / vla::kQRows;
   const KernelAttrs& ka = kernel_attrs<D>();
   if (!ka.ok) return VLA_ATTN_ERR_CUDA;
   const int max_smem = di.max_smem_optin - ka.static_smem;
-  int ring = (max_smem - static_cast<int>(2 * G::kQBytes + vla::kBarrierRegionBytes +
-                                          vla::kAlignSlack)) /
-             static_cast<int>(2 * G::kKVStride);
-  if (ring > vla::kMaxRing) ring = vla::kMaxRing;
+  // K/V ring slots that fit beside qbuf Q buffers per slot and the output
+  // staging.  Two Q buffers per slot (the next round's Q tile loads during
+  // the current round) only when that still leaves a ring of kMinRingQ2.
+  auto ring_for = [&](int qbuf) {
+    const int r = (max_smem - static_cast<int>(2 * qbuf * G::kQBytes + G::kStageBytes +
+                                               vla::kBarrierRegionBytes + vla::kAlignSlack)) /
+                  static_cast<int>(2 * G::kKVStride);
+    return r > vla::kMaxRing ? vla::kMaxRing : r;
+  };
+  constexpr int kMinRingQ2 = 4;
+  int qbuf = vla::kMaxQBuf;
+  int ring = ring_for(qbuf);
+  if (ring < kMinRingQ2) {
+    qbuf = 1;
+    ring = ring_for(qbuf);
+  }
   if (ring < 2) return VLA_ATTN_ERR_DEVICE;
-  const uint32_t smem = vla::smem_bytes_for_ring<D>(ring);
+  const uint32_t smem = vla::smem_bytes_for<D>(ring, qbuf);
 
-  prm.o = static_cast<__nv_bfloat16*>(o);
   prm.B = B;
   prm.N = N;
   prm.H = H;
@@ -340,6 +394,7 @@ int launch(const void* q, void* o, int B, int N, int H, float scale, cudaStream_
   if (units > 0x7FFFFFFFll) return VLA_ATTN_ERR_SHAPE;
   prm.num_units = static_cast<int>(units);
   prm.ring = ring;
+  prm.qbuf = qbuf;
   prm.reuse = (nb <= ring && !prm.stream) ? 1 : 0;
   prm.c = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
   const unsigned long long lim = g_wait_limit_ns.load();
