@@ -368,9 +368,24 @@ __device__ __forceinline__ void gemm_epilogue_loop(const GemmParams& p, uint32_t
   const uint32_t lane_bits = static_cast<uint32_t>(quad * 32) << 16;
   const size_t tile_elems = static_cast<size_t>(kBM) * BN;
   const int tiles = p.tiles_m * p.tiles_n;
+  // The residual of this warp's chunk c of tile (mt, nt) into its buffer, once
+  // the store that last read the buffer is done reading it.
+  auto load_res = [&](const Work& w, int c) {
+    if (lane == 0) {
+      bulk_wait_read<0>();
+      mbar_arrive_expect_tx(bar.res_full(ew), kStageOutBytes);
+      tma_load_2d(buf_s, &p.tm_res, bar.res_full(ew), w.nt * BN + 64 * c, w.mt * kBM + quad * 32);
+    }
+    __syncwarp();
+    rs.pending = true;
+  };
+  const bool res_tiles = p.res != nullptr && p.splits == 1 && set < BN / 64;
   Work wk;
   for (int i = 0; work_at(p, i, wk); ++i) {
     const int buf = i & 1;
+    // The first chunk's residual does not depend on the accumulator: its load
+    // runs while the tile's MMAs do.
+    if (res_tiles) load_res(wk, set);
     if (!wait_bounded(bar.acc_full(buf), (i >> 1) & 1, abort_flag, p.wait_limit_ns, kSiteEpi))
       return;
     tc_fence_after();
@@ -464,19 +479,17 @@ __device__ __forceinline__ void gemm_epilogue_loop(const GemmParams& p, uint32_t
 #pragma unroll 1
     for (int c = set; c < BN / 64; c += 2) {
       const int n0 = n_base + 64 * c;
-      // The store that last read this warp's buffer must be done reading it.
-      if (lane == 0) bulk_wait_read<0>();
-      __syncwarp();
       if (p.res != nullptr) {
-        const uint32_t rb = bar.res_full(ew);
-        if (lane == 0) {
-          mbar_arrive_expect_tx(rb, kStageOutBytes);
-          tma_load_2d(buf_s, &p.tm_res, rb, n0, row0);
-        }
-        rs.pending = true;
-        if (!wait_bounded(rb, rs.issued & 1u, abort_flag, p.wait_limit_ns, kSiteEpi)) return;
+        if (c != set) load_res(wk, c);
+        if (!wait_bounded(bar.res_full(ew), rs.issued & 1u, abort_flag, p.wait_limit_ns,
+                          kSiteEpi))
+          return;
         rs.pending = false;
         ++rs.issued;
+      } else {
+        // The store that last read this warp's buffer must be done reading it.
+        if (lane == 0) bulk_wait_read<0>();
+        __syncwarp();
       }
       uint32_t a[64];
       tmem_ld32(t + 64 * c, reinterpret_cast<uint32_t(&)[32]>(a[0]));
