@@ -861,9 +861,10 @@ __device__ void softmax_role(const AttnParams& p, uint32_t tmem, const Barriers&
                              volatile int* abort_flag, int warp, int lane, uint32_t stage,
                              uint32_t stage_tail) {
   softmax_loop<D>(p, tmem, bar, abort_flag, warp, lane, stage, stage_tail);
-  // This warp's output stores must have read the staging buffer (and
-  // completed) before the CTA ends, on every path out of the loop.
-  if (lane == 0) bulk_wait_all();
+  // This warp's output stores must have read the staging buffer before the
+  // CTA ends, on every path out of the loop (their writes are visible to
+  // whatever follows the grid once it has completed).
+  if (lane == 0) bulk_wait_read<0>();
   __syncwarp();
 }
 

@@ -533,9 +533,10 @@ __device__ __forceinline__ void gemm_epilogue_role(const GemmParams& p, uint32_t
   gemm_epilogue_loop<BN>(p, tmem, bar, abort_flag, warp, lane,
                          staging + static_cast<uint32_t>(ew) * kStageOutBytes, rs);
   // On every way out: a residual load not waited for must land, and every TMA
-  // store of this warp must have finished, before the CTA exits.
+  // store of this warp must have read its staging buffer, before the CTA
+  // exits (the stores' writes are visible once the grid has completed).
   if (rs.pending) wait_drain(bar.res_full(ew), rs.issued & 1u, kDrainLimitNs);
-  if (lane == 0) bulk_wait_all();
+  if (lane == 0) bulk_wait_read<0>();
   __syncwarp();
 }
 
