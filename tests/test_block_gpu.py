@@ -516,3 +516,27 @@ def test_encoder_chain_against_oracle_chain_eager_and_graph():
     check(xs[-1], "graph-replayed encoder chain")
     assert torch.equal(xs[-1], eager), "graph replay differs from the eager run"
     del g
+
+
+@pytest.mark.parametrize("M,K,N,res", [(1, 64, 64, False), (37, 128, 200, True),
+                                       (129, 256, 320, False), (300, 192, 72, True)])
+def test_linear_stores_stay_inside_the_output(M, K, N, res):
+    """The GEMM's output (and residual) move as TMA boxes of 32 rows x 64 columns, which
+    overhang the tensor when M or N is ragged: nothing outside [M, N] may be written.  The
+    output is a view into a larger buffer whose guards hold a sentinel; they must be
+    unchanged and the output must match the oracle."""
+    import vit_self_attention_b200 as vab
+    x, w, b = linear_inputs(M, K, N, 5100 + M + K + N)
+    r = si.normal_bf16(5400 + M, (M, N)) if res else None
+    n_y = M * N
+    guard = 8 * 1024  # elements (16 KB) on each side, 16-byte aligned
+    sentinel = 0x7FA5
+    big = torch.full((guard + n_y + guard,), sentinel, dtype=torch.int16, device="cuda")
+    y = big[guard:guard + n_y].view(torch.bfloat16).view(M, N)
+    vab.linear(dev(x), dev(w), dev(b), dev(r) if res else None, out=y)
+    torch.cuda.synchronize()
+    assert bool((big[:guard] == sentinel).all()), "written before the output"
+    assert bool((big[guard + n_y:] == sentinel).all()), "written after the output"
+    assert_close_bf16(f64(y), oracle.linear_bf16(x, w, b, r),
+                      f"guarded linear M={M} K={K} N={N} res={res}",
+                      mag=residual_magnitude(x, w, b, r))

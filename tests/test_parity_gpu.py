@@ -338,3 +338,30 @@ def test_host_entry_rejects_short_device_buffers_before_copying():
         assert st == vab.ERR_MEMORY
     finally:
         cudart.cudaFree(raw)
+
+
+@pytest.mark.parametrize("B,N,H,d", [(1, 1, 1, 64), (1, 33, 2, 64), (2, 97, 3, 64), (1, 577, 2, 64),
+                                     (1, 50, 2, 72), (2, 113, 3, 72)])
+def test_output_stores_stay_inside_the_output(B, N, H, d):
+    """The output leaves through TMA stores of 32-row boxes, which overhang the tensor at the
+    last rows of every image when N is not a multiple of 32: nothing outside [B, N, H, d] may
+    be written.  The output is a view into a larger buffer whose guard regions before and
+    after it hold a sentinel; they must be unchanged and the output must match the oracle."""
+    import vit_self_attention_b200 as vab
+    bits = si.packed_qkv(B, N, H, d, seed=4100 + 7 * N + d)
+    scale = 1.0 / math.sqrt(d)
+    want = oracle.attention_packed_bf16(bits, scale)
+    qkv = device_qkv(bits)
+    n_o = B * N * H * d
+    guard = 8 * 1024  # elements (16 KB) on each side, 16-byte aligned
+    sentinel = 0x7FA5
+    big = torch.full((guard + n_o + guard,), sentinel, dtype=torch.int16, device="cuda")
+    o = big[guard:guard + n_o]
+    base = qkv.data_ptr()
+    hd = H * d * 2
+    vab.vla_attn_fwd(base, base + hd, base + 2 * hd, o.data_ptr(), B, N, H, d, scale)
+    torch.cuda.synchronize()
+    assert bool((big[:guard] == sentinel).all()), "written before the output"
+    assert bool((big[guard + n_o:] == sentinel).all()), "written after the output"
+    got = o.view(torch.bfloat16).float().cpu().numpy().astype(np.float64).reshape(B, N, H, d)
+    assert_parity(got, want, f"guarded B={B} N={N} H={H} d={d}")
