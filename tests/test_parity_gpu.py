@@ -81,13 +81,17 @@ def test_longest_sequence_sampled_rows():
                                      (160, 1, 197, 64), (10, 16, 257, 64), (12, 13, 577, 64),
                                      (75, 2, 577, 72), (1, 1, 577, 64), (148, 1, 129, 72),
                                      (300, 1, 50, 64), (10, 16, 1025, 64), (149, 1, 577, 64),
-                                     (297, 1, 300, 64), (157, 1, 600, 72)])
+                                     (297, 1, 300, 64), (157, 1, 600, 72), (10, 16, 700, 64),
+                                     (10, 16, 500, 72), (10, 16, 512, 64), (10, 16, 448, 72)])
 def test_schedules(B, H, N, d):
     """Whole-head work units (B*H >= #SMs), per-round units (fewer heads, more tiles than
-    SMs; includes K/V streaming at N > 768 / d=72 N > 560), single-tile units (all tiles
-    fit on the SMs), persistent multi-unit CTAs, and stream mode (whole heads with an odd
-    tile count: tiles paired across head boundaries, a lone last tile on CTAs with an odd
-    tile total, K/V streamed, with and without the long-sequence ring wrap)."""
+    SMs; K/V streamed when a head's blocks do not fit the ring), single-tile units (all
+    tiles fit on the SMs), persistent multi-unit CTAs, and stream mode (whole heads with an
+    odd tile count: tiles paired across head boundaries, a lone last tile on CTAs with an
+    odd tile total, K/V streamed, with and without the long-sequence ring wrap).  The
+    shared-memory plans: two Q buffers with a ring of 4 and the output staging (N=512 /
+    448: a head's K/V resident), and whole heads of 6 (d=64, N=700) or 5 (d=72, N=500)
+    key blocks, resident only in the longer ring without the staging (row stores)."""
     bits = si.packed_qkv(B, N, H, d, seed=90000 + B * 7 + H * 3 + N + d)
     scale = 1.0 / math.sqrt(d)
     want = oracle.attention_packed_bf16(bits, scale)
@@ -341,11 +345,12 @@ def test_host_entry_rejects_short_device_buffers_before_copying():
 
 
 @pytest.mark.parametrize("B,N,H,d", [(1, 1, 1, 64), (1, 33, 2, 64), (2, 97, 3, 64), (1, 577, 2, 64),
-                                     (1, 50, 2, 72), (2, 113, 3, 72)])
+                                     (1, 50, 2, 72), (2, 113, 3, 72), (10, 700, 16, 64)])
 def test_output_stores_stay_inside_the_output(B, N, H, d):
     """The output leaves through TMA stores of 32-row boxes, which overhang the tensor at the
-    last rows of every image when N is not a multiple of 32: nothing outside [B, N, H, d] may
-    be written.  The output is a view into a larger buffer whose guard regions before and
+    last rows of every image when N is not a multiple of 32 (or, for whole heads resident
+    only without the staging, N=700, through 16-byte row stores): nothing outside
+    [B, N, H, d] may be written.  The output is a view into a larger buffer whose guard regions before and
     after it hold a sentinel; they must be unchanged and the output must match the oracle."""
     import vit_self_attention_b200 as vab
     bits = si.packed_qkv(B, N, H, d, seed=4100 + 7 * N + d)

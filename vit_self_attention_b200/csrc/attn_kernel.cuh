@@ -24,7 +24,9 @@
 //               columns, O rescaled in tensor memory only when the running
 //               maximum grows by more than 2^8, epilogue O / l -> bf16 into
 //               a per-warp shared-memory buffer written out by one TMA store
-//               of the warp's 32 rows (whole 128-byte rows per transaction).
+//               of the warp's 32 rows (whole 128-byte rows per transaction),
+//               or, where the staging's space is needed for a longer K/V ring,
+//               by 16-byte row stores.
 //   warp 3      idle.
 //
 // Schedule.  A round holds up to two 128-row Q tiles, one per Q slot and
@@ -165,13 +167,14 @@ struct AttnParams {
                            // (whole heads with an odd tile count), K/V streamed
   int qbuf;                // Q buffers per slot (1 or 2): with 2 the next round's Q tile
                            // loads while the current round runs
+  __nv_bfloat16* o;        // [B, N, H, d] (the row stores of the kernel without staging)
 };
 
 template <int D>
-__host__ __device__ constexpr uint32_t smem_bytes_for(int ring, int qbuf) {
+__host__ __device__ constexpr uint32_t smem_bytes_for(int ring, int qbuf, bool stage_out) {
   return 2u * static_cast<uint32_t>(qbuf) * Geom<D>::kQBytes +
-         2u * static_cast<uint32_t>(ring) * Geom<D>::kKVStride + Geom<D>::kStageBytes +
-         kBarrierRegionBytes + kAlignSlack;
+         2u * static_cast<uint32_t>(ring) * Geom<D>::kKVStride +
+         (stage_out ? Geom<D>::kStageBytes : 0u) + kBarrierRegionBytes + kAlignSlack;
 }
 
 struct Barriers {
@@ -732,12 +735,13 @@ struct OutRow {
   float inv_l;
 };
 
-// O / l -> bf16 for this warp's 32 rows through its shared-memory staging
-// buffer (128-byte swizzle: 16-byte chunk t of row r at chunk t ^ (r mod 8),
-// so the eight rows of a store phase hit distinct banks), then one TMA
-// store of the 32 x d box; rows past N fall outside the tensor and are not
-// written.  The tensor-memory loads are warp-collective.
-template <int D>
+// O / l -> bf16 for this warp's 32 rows: with kStageOut through its
+// shared-memory staging buffer (128-byte swizzle: 16-byte chunk t of row r
+// at chunk t ^ (r mod 8), so the eight rows of a store phase hit distinct
+// banks), then one TMA store of the 32 x d box, rows past N falling outside
+// the tensor; without, each thread's row by 16-byte stores.  The
+// tensor-memory loads are warp-collective.
+template <int D, bool kStageOut>
 __device__ __forceinline__ void store_output(const AttnParams& p, uint32_t tO, const OutRow& r,
                                              uint32_t stage, uint32_t stage_tail, int lane) {
   using G = Geom<D>;
@@ -746,6 +750,26 @@ __device__ __forceinline__ void store_output(const AttnParams& p, uint32_t tO, c
   uint32_t ot[16];
   if (G::DP > 64) tmem_ld16(tO + 64, ot);
   if (r.row0 >= p.N) return;  // warp-uniform: no row of this warp is a token
+  if constexpr (!kStageOut) {
+    // 16-byte stores of this thread's row (rows past N are not written).
+    const int row = r.row0 + (lane & 31);
+    if (row < p.N) {
+      uint4* d4 = reinterpret_cast<uint4*>(
+          p.o + ((static_cast<size_t>(r.b) * p.N + row) * p.H + r.h) * D);
+#pragma unroll
+      for (int t = 0; t < D / 8; ++t) {
+        float v[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          const int ch = 8 * t + e;
+          v[e] = __uint_as_float(ch < 64 ? ob[ch] : ot[ch - 64]) * r.inv_l;
+        }
+        d4[t] = make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]),
+                           pack_bf16x2(v[4], v[5]), pack_bf16x2(v[6], v[7]));
+      }
+    }
+    return;
+  }
   // The previous store from this buffer must have finished reading it.
   if (lane == 0) bulk_wait_read<0>();
   __syncwarp();
@@ -778,7 +802,7 @@ __device__ __forceinline__ void store_output(const AttnParams& p, uint32_t tO, c
 // (after the previous P V has finished with the P columns) store P; after a
 // round's last block, O / l of its Q tile to the output.
 
-template <int D>
+template <int D, bool kStageOut>
 __device__ void softmax_loop(const AttnParams& p, uint32_t tmem, const Barriers& bar,
                              volatile int* abort_flag, int warp, int lane, uint32_t stage,
                              uint32_t stage_tail) {
@@ -852,15 +876,15 @@ __device__ void softmax_loop(const AttnParams& p, uint32_t tmem, const Barriers&
     if (!wait_pv()) return;
     VLA_TRACE_EVENT(kTrSoftEpi, s, 0);
     const OutRow r{x.b(s), x.h(s), x.tile(s) * kQRows + quad * 32, 1.0f / st.l_run};
-    store_output<D>(p, tO, r, stage, stage_tail, lane);
+    store_output<D, kStageOut>(p, tO, r, stage, stage_tail, lane);
   }
 }
 
-template <int D>
+template <int D, bool kStageOut>
 __device__ void softmax_role(const AttnParams& p, uint32_t tmem, const Barriers& bar,
                              volatile int* abort_flag, int warp, int lane, uint32_t stage,
                              uint32_t stage_tail) {
-  softmax_loop<D>(p, tmem, bar, abort_flag, warp, lane, stage, stage_tail);
+  softmax_loop<D, kStageOut>(p, tmem, bar, abort_flag, warp, lane, stage, stage_tail);
   // This warp's output stores must have read the staging buffer before the
   // CTA ends, on every path out of the loop (their writes are visible to
   // whatever follows the grid once it has completed).
@@ -869,7 +893,9 @@ __device__ void softmax_role(const AttnParams& p, uint32_t tmem, const Barriers&
 }
 
 // ------------------------------------------------------------ kernel
-template <int D>
+// kStageOut: the output through shared-memory staging and TMA stores (else
+// 16-byte row stores, leaving the staging's space to the K/V ring).
+template <int D, bool kStageOut>
 __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_constant__ AttnParams p) {
   using G = Geom<D>;
   extern __shared__ uint8_t smem_raw[];
@@ -879,7 +905,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
   const uint32_t sK = sQ + 2 * p.qbuf * G::kQBytes;
   const uint32_t sV = sK + p.ring * G::kKVStride;
   const uint32_t sStage = sV + p.ring * G::kKVStride;
-  const uint32_t sBar = sStage + G::kStageBytes;
+  const uint32_t sBar = sStage + (kStageOut ? G::kStageBytes : 0u);
   uint8_t* bar_generic = smem_raw + (sBar - raw);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_generic + 8 * kNumBarriers);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(bar_generic + 8 * kNumBarriers + 4);
@@ -915,11 +941,11 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
   if (warp == kLoadWarp && lane == 0) {
     prefetch_tmap(&p.tm_q);
     prefetch_tmap(&p.tm_kv);
-    prefetch_tmap(&p.tm_o);
+    if (kStageOut) prefetch_tmap(&p.tm_o);
     if (G::kHasTail) {
       prefetch_tmap(&p.tm_q_tail);
       prefetch_tmap(&p.tm_kv_tail);
-      prefetch_tmap(&p.tm_o_tail);
+      if (kStageOut) prefetch_tmap(&p.tm_o_tail);
     }
   }
   if (warp == kMmaWarp) {
@@ -943,7 +969,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
     __syncwarp();
   } else if (warp >= kSoftmaxWarp0) {
     const int ws = warp - kSoftmaxWarp0;  // staging buffer of this warp
-    softmax_role<D>(p, tmem, bar, abort_flag, warp, lane, sStage + ws * G::kStageWarp,
+    softmax_role<D, kStageOut>(p, tmem, bar, abort_flag, warp, lane, sStage + ws * G::kStageWarp,
                     sStage + 8 * G::kStageWarp + ws * G::kStageTailWarp);
     __syncwarp();
   }

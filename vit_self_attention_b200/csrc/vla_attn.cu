@@ -69,8 +69,8 @@ struct DeviceInfo {
   bool supported = false;
   int sm_count = 0;
   int max_smem_optin = 0;
-  int attr64 = 0;  // dynamic shared memory limit set on the d = 64 kernel (0 = not yet)
-  int attr72 = 0;
+  int attr[2][2] = {{0, 0}, {0, 0}};  // dynamic shared memory limit set per kernel
+                                      // [d = 72][staging] (0 = not yet)
 };
 
 std::mutex g_dev_mutex;
@@ -141,13 +141,13 @@ int host_pipe(int dev, HostPipe** out) {
 }
 
 // Raises the kernel's dynamic shared-memory limit to at least `smem` bytes.
-template <int D>
+template <int D, bool kStageOut>
 int ensure_smem_attr(int dev, int smem) {
   std::lock_guard<std::mutex> lock(g_dev_mutex);
-  int& cur = (D == 64) ? g_dev[dev].attr64 : g_dev[dev].attr72;
+  int& cur = g_dev[dev].attr[D == 72 ? 1 : 0][kStageOut ? 1 : 0];
   if (cur < smem) {
-    if (cudaFuncSetAttribute(vla::attn_fwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             smem) != cudaSuccess)
+    if (cudaFuncSetAttribute(vla::attn_fwd_kernel<D, kStageOut>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
       return VLA_ATTN_ERR_CUDA;
     cur = smem;
   }
@@ -168,7 +168,7 @@ const KernelAttrs& kernel_attrs() {
   static std::once_flag once;
   std::call_once(once, [] {
     cudaFuncAttributes fa{};
-    if (cudaFuncGetAttributes(&fa, vla::attn_fwd_kernel<D>) == cudaSuccess) {
+    if (cudaFuncGetAttributes(&fa, vla::attn_fwd_kernel<D, true>) == cudaSuccess) {
       a.static_smem = static_cast<int>(fa.sharedSizeBytes);
       a.regs = fa.numRegs;
       a.ok = true;
@@ -355,24 +355,43 @@ int launch(const void* q, void* o, int B, int N, int H, float scale, cudaStream_
   const KernelAttrs& ka = kernel_attrs<D>();
   if (!ka.ok) return VLA_ATTN_ERR_CUDA;
   const int max_smem = di.max_smem_optin - ka.static_smem;
-  // K/V ring slots that fit beside qbuf Q buffers per slot and the output
-  // staging.  Two Q buffers per slot (the next round's Q tile loads during
-  // the current round) only when that still leaves a ring of kMinRingQ2.
-  auto ring_for = [&](int qbuf) {
-    const int r = (max_smem - static_cast<int>(2 * qbuf * G::kQBytes + G::kStageBytes +
+  // Shared memory: Q buffers (qbuf per slot), the K/V ring, and the output
+  // staging when the output leaves by TMA stores (stage_out).  The default is
+  // staging with two Q buffers (the next round's Q tile loads during the
+  // current round) while that leaves a ring of four blocks, else one.  When a
+  // head's K/V blocks fit a ring only without the staging (whole-head units
+  // with 5 or 6 blocks), the output goes by row stores instead and the head's
+  // K/V stay resident for all its rounds.
+  auto ring_for = [&](int qbuf, bool staged) {
+    const int r = (max_smem - static_cast<int>(2 * qbuf * G::kQBytes +
+                                               (staged ? G::kStageBytes : 0u) +
                                                vla::kBarrierRegionBytes + vla::kAlignSlack)) /
                   static_cast<int>(2 * G::kKVStride);
     return r > vla::kMaxRing ? vla::kMaxRing : r;
   };
+  const long long heads_total = static_cast<long long>(B) * H;
+  const bool whole_heads = heads_total >= di.sm_count;
+  const bool streams = whole_heads && nq > 1 && (nq & 1);
   constexpr int kMinRingQ2 = 4;
+  bool stage_out = true;
   int qbuf = vla::kMaxQBuf;
-  int ring = ring_for(qbuf);
+  int ring = ring_for(qbuf, true);
   if (ring < kMinRingQ2) {
     qbuf = 1;
-    ring = ring_for(qbuf);
+    ring = ring_for(qbuf, true);
+  }
+  if (whole_heads && !streams && nb > ring) {
+    if (nb <= ring_for(1, true)) {
+      qbuf = 1;
+      ring = ring_for(1, true);
+    } else if (nb <= ring_for(1, false)) {
+      stage_out = false;
+      qbuf = 1;
+      ring = ring_for(1, false);
+    }
   }
   if (ring < 2) return VLA_ATTN_ERR_DEVICE;
-  const uint32_t smem = vla::smem_bytes_for<D>(ring, qbuf);
+  const uint32_t smem = vla::smem_bytes_for<D>(ring, qbuf, stage_out);
 
   prm.B = B;
   prm.N = N;
@@ -395,13 +414,15 @@ int launch(const void* q, void* o, int B, int N, int H, float scale, cudaStream_
   prm.num_units = static_cast<int>(units);
   prm.ring = ring;
   prm.qbuf = qbuf;
+  prm.o = static_cast<__nv_bfloat16*>(o);
   prm.reuse = (nb <= ring && !prm.stream) ? 1 : 0;
   prm.c = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
   const unsigned long long lim = g_wait_limit_ns.load();
   prm.wait_limit_ns = lim == 0 ? kDefaultWaitLimitNs : lim;
   prm.test_stall = g_test_stall.load();
 
-  rc = ensure_smem_attr<D>(dev, static_cast<int>(smem));
+  rc = stage_out ? ensure_smem_attr<D, true>(dev, static_cast<int>(smem))
+                 : ensure_smem_attr<D, false>(dev, static_cast<int>(smem));
   if (rc != VLA_ATTN_OK) return rc;
 
   const int grid = static_cast<int>(units < di.sm_count ? units : di.sm_count);
@@ -412,7 +433,9 @@ int launch(const void* q, void* o, int B, int N, int H, float scale, cudaStream_
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
   set_dependent_launch(&cfg, attr);
-  if (cudaLaunchKernelEx(&cfg, vla::attn_fwd_kernel<D>, prm) != cudaSuccess) {
+  const cudaError_t le = stage_out ? cudaLaunchKernelEx(&cfg, vla::attn_fwd_kernel<D, true>, prm)
+                                   : cudaLaunchKernelEx(&cfg, vla::attn_fwd_kernel<D, false>, prm);
+  if (le != cudaSuccess) {
     (void)cudaGetLastError();
     return VLA_ATTN_ERR_CUDA;
   }
