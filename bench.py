@@ -106,10 +106,14 @@ _REASON_BITS = {
 
 
 class ClockSampler:
-    """Samples SM clock and throttle reasons through NVML while the timed region runs."""
+    """Samples SM clock and throttle reasons through NVML from before the warm-up to the
+    end of the timed region; the summary keeps the samples taken inside the timed region
+    (host times t0..t1 set by mark_start / mark_end)."""
 
-    def __init__(self, device_index: int, period_s: float = 0.001):
-        self.samples: list[tuple[int, int]] = []
+    def __init__(self, device_index: int, period_s: float = 0.0002):
+        self.samples: list[tuple[float, int, int]] = []
+        self._t0 = None
+        self._t1 = None
         self.max_mhz = None
         self._stop = threading.Event()
         self._period = period_s
@@ -129,9 +133,10 @@ class ClockSampler:
         nv = self._nvml
         while not self._stop.is_set():
             try:
+                t = time.perf_counter()
                 mhz = int(nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM))
                 reasons = int(nv.nvmlDeviceGetCurrentClocksEventReasons(self._h))
-                self.samples.append((mhz, reasons))
+                self.samples.append((t, mhz, reasons))
             except Exception:
                 pass
             time.sleep(self._period)
@@ -146,12 +151,26 @@ class ClockSampler:
         if self._ok:
             self._t.join()
 
+    def mark_start(self):
+        self._t0 = time.perf_counter()
+
+    def mark_end(self):
+        self._t1 = time.perf_counter()
+
     def summary(self) -> dict | None:
         if not self._ok or not self.samples:
             return None
-        mhz = [m for m, _ in self.samples]
+        t0 = self._t0 if self._t0 is not None else float("-inf")
+        t1 = self._t1 if self._t1 is not None else float("inf")
+        inside = [(m, r) for t, m, r in self.samples if t0 <= t <= t1]
+        if not inside:  # a region shorter than one NVML query: the last sample before it
+            before = [(m, r) for t, m, r in self.samples if t < t0]
+            inside = before[-1:]
+        if not inside:
+            return None
+        mhz = [m for m, _ in inside]
         seen = 0
-        for _, r in self.samples:
+        for _, r in inside:
             seen |= r
         names = sorted(n for bit, n in _REASON_BITS.items() if seen & bit and n != "gpu_idle")
         return {"sm_mhz": float(statistics.median(mhz)), "sm_max_mhz": self.max_mhz,
@@ -269,21 +288,22 @@ def run_ours(args, rank: int, world: int, local_rank: int) -> None:
         if world > 1:
             dist.barrier()
 
-    for _ in range(max(3, args.warmup)):
-        step()
-    torch.cuda.synchronize()
-
-    launches0 = vab.vla_attn_launch_count()
     ev0 = torch.cuda.Event(enable_timing=True)
     ev1 = torch.cuda.Event(enable_timing=True)
     with ClockSampler(local_rank) as clocks:
+        for _ in range(max(3, args.warmup)):
+            step()
+        torch.cuda.synchronize()
+        launches0 = vab.vla_attn_launch_count()
         barrier()
         torch.cuda.synchronize()
+        clocks.mark_start()
         ev0.record(stream)
         for _ in range(args.steps):
             step()
         ev1.record(stream)
         torch.cuda.synchronize()
+        clocks.mark_end()
         barrier()
     launches = vab.vla_attn_launch_count() - launches0
     ms = ev0.elapsed_time(ev1)

@@ -47,13 +47,20 @@ def test_clock_summary_reasons_and_median():
     bench = _bench()
     cs = bench.ClockSampler.__new__(bench.ClockSampler)
     cs._ok, cs.max_mhz = True, 1965
-    cs.samples = [(1965, 0x1), (1965, 0x4), (1845, 0x4 | 0x8), (1965, 0)]
+    cs._t0, cs._t1 = 10.0, 11.0
+    # (host time, MHz, reasons): samples before and after the timed region are dropped.
+    cs.samples = [(9.0, 1200, 0x20), (10.1, 1965, 0x1), (10.2, 1965, 0x4),
+                  (10.5, 1845, 0x4 | 0x8), (10.9, 1965, 0), (11.5, 900, 0x40)]
     s = cs.summary()
     assert s["sm_mhz"] == 1965.0 and s["sm_max_mhz"] == 1965 and s["sm_mhz_min"] == 1845
     assert s["reasons"] == ["hw_slowdown", "sw_power_cap"]  # idle is not a throttle reason
     assert s["samples"] == 4
+    # A region shorter than one query: the last sample before it stands in.
+    cs._t0, cs._t1 = 9.5, 9.6
+    s = cs.summary()
+    assert s["samples"] == 1 and s["sm_mhz"] == 1200.0
     cs.samples = []
     assert cs.summary() is None
     cs._ok = False
-    cs.samples = [(1965, 0)]
+    cs.samples = [(10.5, 1965, 0)]
     assert cs.summary() is None
