@@ -198,11 +198,13 @@ int vla_layernorm_fwd(const void* x, const void* gamma, const void* beta, void* 
  *   K, N     multiples of 8.  All pointers 16-byte aligned.
  *   workspace, workspace_bytes  caller-owned device scratch (NULL with 0
  *            allowed).  When the output has too few 128-row tiles to fill the
- *            SMs, the K range is split and the parts' fp32 partial sums and
- *            per-tile arrival counters go here (the counters are cleared by a
- *            memset enqueued before the kernel); a shape is split only if its
- *            partial sums fit, otherwise it runs unsplit (same result up to
- *            fp32 summation order).  vla_linear_workspace_bytes() is enough
+ *            SMs and K is long enough for the split to pay (in practice K of
+ *            several thousand and more with a few tiles; none of the encoder
+ *            shapes), the K range is split and the parts' fp32 partial sums
+ *            and per-tile arrival counters go here (the counters are cleared
+ *            by a memset enqueued before the kernel); a shape is split only if
+ *            its partial sums fit, otherwise it runs unsplit (same result up
+ *            to fp32 summation order).  vla_linear_workspace_bytes() is enough
  *            for every split the library chooses.  The library allocates
  *            nothing.  Calls that share a workspace must be ordered on one
  *            stream.

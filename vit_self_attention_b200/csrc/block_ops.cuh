@@ -223,9 +223,14 @@ struct LinearPlan {
 // Tile width: the fewest waves of tiles over the SMs weighted by a tile's cost,
 // its MMA time (proportional to BN) plus its 128-row tile of x (loaded whatever
 // BN is), wider tiles on ties (more reuse per byte loaded).  Split K when the
-// tiles fill at most a quarter of the SMs (with more tiles, adding the parts'
-// partial sums costs more than the split gains) and
-// the caller's workspace holds the partial sums.
+// tiles fill at most a quarter of the SMs, the caller's workspace holds the
+// partial sums, and the main-loop time the split saves exceeds its fixed cost:
+// the counters' memset ahead of the launch, which also forgoes the overlap with
+// the previous kernel, and the partial sums' round trip, about 7 us (measured:
+// split calls of the 50- to 591-token encoder shapes, K <= 4096, ran at twice
+// the time of the same shapes unsplit).
+constexpr long long kSplitFixedCycles = 14000;
+
 LinearPlan plan_linear(int M, int K, int N, int sm_count, size_t workspace_bytes) {
   LinearPlan pl;
   pl.tiles_m = (M + vla::gemm::kBM - 1) / vla::gemm::kBM;
@@ -243,6 +248,8 @@ LinearPlan plan_linear(int M, int K, int N, int sm_count, size_t workspace_bytes
   pl.tiles_n = (N + pl.bn - 1) / pl.bn;
   const long long tiles = static_cast<long long>(pl.tiles_m) * pl.tiles_n;
   pl.ksteps_per_split = pl.ksteps;
+  // Cycles per k-step of one tile: its MMAs or its loads, whichever is longer.
+  const long long step = std::max(2ll * pl.bn, 128ll + pl.bn);
   if (4 * tiles <= sm_count && pl.ksteps >= 8) {
     int splits = static_cast<int>(sm_count / tiles);
     splits = std::min(splits, pl.ksteps / 4);
@@ -252,6 +259,8 @@ LinearPlan plan_linear(int M, int K, int N, int sm_count, size_t workspace_bytes
       const int used = (pl.ksteps + per - 1) / per;  // no empty part
       const size_t need = static_cast<size_t>(used) * tiles * vla::gemm::kBM * pl.bn * 4u +
                           static_cast<size_t>(tiles) * 4u * sizeof(unsigned int);
+      const long long saved = static_cast<long long>(pl.ksteps - per) * step;
+      if (saved <= kSplitFixedCycles) break;  // fewer parts save less
       if (need <= workspace_bytes) {
         pl.splits = used;
         pl.ksteps_per_split = per;
