@@ -9,6 +9,7 @@ batch.  Prints ONE JSON line (rank 0).
   python bench.py --configs     # per-config report (one JSON line per item, 1 GPU)
   python bench.py --block       # LayerNorm / linear layers, whole encoder layers and encoders
   python bench.py --linear M,K,N   # one linear layer of that shape
+  python bench.py --layer WORKLOAD # one encoder layer, stage by stage
 
 Under torchrun every rank runs the same per-GPU batch on its own GPU (weak
 scaling, no collective on the data path); the elapsed time is the max over
@@ -700,6 +701,76 @@ def run_block(args) -> None:
         torch.cuda.empty_cache()
 
 
+def run_layer(args) -> None:
+    """One whole pre-norm encoder layer of a named workload (LN1 -> qkv -> attention ->
+    output projection + residual -> LN2 -> fc1 + GELU -> fc2 + residual), seeded weights
+    and activations, launched eagerly stage by stage: three warm layers, then ten timed
+    ones with CUDA events around every stage (one JSON line of per-stage medians).  Its
+    launches in stream order are what an ncu launch list of one layer shows."""
+    import math as _m
+
+    import torch
+
+    import vit_self_attention_b200 as vab
+
+    names = {c.name: c for c in list(si.ENCODER_WORKLOADS) + [si.VIT_L14_336PX_B256]}
+    if args.layer not in names:
+        raise SystemExit(f"--layer: one of {sorted(names)}")
+    c = names[args.layer]
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    W = c.H * c.d
+    F = {768: 3072, 1024: 4096, 1152: 4304}[W]
+
+    def t_(shape, mean=0.0, std=1.0, seed=1):
+        b = si.normal_bf16(seed, shape, mean, std)
+        return torch.from_numpy(b.view(np.int16)).to(dev).view(torch.bfloat16)
+
+    g, be = t_((W,), 1.0, 0.1, 12), t_((W,), 0.0, 0.1, 13)
+    wq, bq = t_((3 * W, W), 0.0, 1.0 / _m.sqrt(W), 14), t_((3 * W,), 0.0, 0.1, 15)
+    wo, bo = t_((W, W), 0.0, 1.0 / _m.sqrt(W), 16), t_((W,), 0.0, 0.1, 17)
+    g2, be2 = t_((W,), 1.0, 0.1, 18), t_((W,), 0.0, 0.1, 19)
+    w1, b1 = t_((F, W), 0.0, 1.0 / _m.sqrt(W), 20), t_((F,), 0.0, 0.1, 21)
+    w2, b2 = t_((W, F), 0.0, 1.0 / _m.sqrt(F), 22), t_((W,), 0.0, 0.1, 23)
+    x = t_((c.B, c.N, W), 0.0, 1.0, 11)
+    xn = torch.empty_like(x)
+    qkv = torch.empty((c.B, c.N, 3 * W), dtype=torch.bfloat16, device=dev)
+    o = torch.empty((c.B, c.N, c.H, c.d), dtype=torch.bfloat16, device=dev)
+    y = torch.empty_like(x)
+    a = torch.empty((c.B, c.N, F), dtype=torch.bfloat16, device=dev)
+    y2 = torch.empty_like(x)
+    ws = torch.empty(vab.vla_linear_workspace_bytes(), dtype=torch.uint8, device=dev)
+    stages = [
+        ("layernorm_1", lambda: vab.layernorm(x, g, be, 1e-6, out=xn)),
+        ("qkv_linear", lambda: vab.linear(xn, wq, bq, out=qkv, workspace=ws)),
+        ("attention", lambda: vab.attention(qkv.view(c.B, c.N, 3, c.H, c.d), c.scale, out=o)),
+        ("out_linear_residual",
+         lambda: vab.linear(o.view(c.B, c.N, W), wo, bo, x, out=y, workspace=ws)),
+        ("layernorm_2", lambda: vab.layernorm(y, g2, be2, 1e-6, out=xn)),
+        ("fc1_gelu", lambda: vab.linear_gelu(xn, w1, b1, out=a, workspace=ws)),
+        ("fc2_residual", lambda: vab.linear(a, w2, b2, y, out=y2, workspace=ws)),
+    ]
+    for _ in range(3):
+        for _, f in stages:
+            f()
+    torch.cuda.synchronize()
+    times = {n: [] for n, _ in stages}
+    for _ in range(10):
+        evs = [torch.cuda.Event(enable_timing=True) for _ in range(len(stages) + 1)]
+        evs[0].record()
+        for i, (_, f) in enumerate(stages):
+            f()
+            evs[i + 1].record()
+        evs[-1].synchronize()
+        for i, (n, _) in enumerate(stages):
+            times[n].append(evs[i].elapsed_time(evs[i + 1]) * 1e3)
+    med = {n: statistics.median(v) for n, v in times.items()}
+    total = sum(med.values())
+    print(json.dumps({"mode": "layer", "workload": c.name, "tokens": c.B * c.N,
+                      "stage_us": med, "layer_us": total,
+                      "share": {n: v / total for n, v in med.items()}}), flush=True)
+
+
 def run_linear(args) -> None:
     """One linear layer y = x w^T + bias (+ a residual, or GELU) on an (M, K, N) shape with
     seeded bf16 operands: five warm calls, then the median of 20 CUDA-event timed calls
@@ -769,6 +840,8 @@ def main() -> None:
                     help="per-config report instead of the benchmark line (1 GPU)")
     ap.add_argument("--block", action="store_true",
                     help="the layers around attention, whole encoder layers and encoders (1 GPU)")
+    ap.add_argument("--layer", default=None, metavar="WORKLOAD",
+                    help="one whole encoder layer of a workload, stage by stage (1 GPU)")
     ap.add_argument("--linear", default=None, metavar="M,K,N[,bias|res|gelu]",
                     help="time one linear layer y = x w^T + bias (+ residual, or GELU) of this "
                          "shape (1 GPU)")
@@ -781,6 +854,9 @@ def main() -> None:
         return
     if args.linear:
         run_linear(args)
+        return
+    if args.layer:
+        run_layer(args)
         return
 
     if "WORLD_SIZE" not in os.environ and args.gpus > 1:
