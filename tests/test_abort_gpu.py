@@ -19,10 +19,10 @@ from gpu_helpers import assert_parity, needs_gpu, run_cuda
 pytestmark = [pytest.mark.gpu, needs_gpu]
 
 # Device status sites (first timed-out wait): producer 1-3, MMA issuers
-# 11-15, softmax 21-22, drains 31, the testing hook's wait 41.  The hook's
+# 11-16, softmax 21-22, drains 31, the testing hook's wait 41.  The hook's
 # wait normally runs out first; a role that started waiting at about the
 # same time may win the race to record its site.
-KNOWN_SITES = {1, 2, 3, 11, 12, 13, 14, 15, 21, 22, 31, 41}
+KNOWN_SITES = {1, 2, 3, 11, 12, 13, 14, 15, 16, 21, 22, 31, 41}
 
 
 @pytest.mark.parametrize("name", ["vit_b16_224px_3views", "siglip_so400m14_224px_2views"])

@@ -82,7 +82,7 @@ constexpr int kThreads = 384;
 constexpr int kMaxRing = 6;
 constexpr uint32_t kTmemCols = 512;
 constexpr int kMaxQBuf = 2;  // Q buffers per slot
-constexpr int kNumBarriers = 16 + 4 * kMaxRing + 3;
+constexpr int kNumBarriers = 16 + 4 * kMaxRing + 5;
 constexpr uint32_t kBarrierRegionBytes = 512;  // barriers + tmem address + abort flag
 constexpr uint32_t kAlignSlack = 1024;
 constexpr unsigned long long kDrainLimitNs = 100000000ull;
@@ -91,6 +91,7 @@ constexpr unsigned long long kDrainLimitNs = 100000000ull;
 enum : int {
   kSiteLoadQ = 1, kSiteLoadK = 2, kSiteLoadV = 3,
   kSiteMmaQ = 11, kSiteMmaK = 12, kSiteMmaV = 13, kSiteMmaP = 14, kSiteMmaFree = 15,
+  kSiteMmaPvIssued = 16,
   kSiteSoftS = 21, kSiteSoftO = 22,
   kSiteDrain = 31,
   kSiteTestStall = 41,
@@ -193,6 +194,8 @@ struct Barriers {
   __device__ uint32_t drain(int i) const { return base + 8u * (16 + 4 * kMaxRing + i); }
   // Never arrived at: the testing hook's wait runs out on it.
   __device__ uint32_t never() const { return base + 8u * (16 + 4 * kMaxRing + 2); }
+  // One phase per P V group issued (not completed) for slot s.
+  __device__ uint32_t pv_issued(int s) const { return base + 8u * (16 + 4 * kMaxRing + 3 + s); }
 };
 
 // Bounded wait for the phase of `bar` with the given parity, executed by a
@@ -456,6 +459,7 @@ __device__ void mma_role(const AttnParams& p, uint32_t tmem, uint32_t sQ, uint32
   uint32_t nf0 = 0, nf1 = 0;  // s_free phases consumed per slot
   uint32_t np0 = 0, np1 = 0;  // p_full phases consumed per slot
   RingPos pos{0, 0u};         // ring position of the next unit / round's first K/V event
+  uint32_t npv0 = 0, npv1 = 0;  // score warp: P V groups of each slot in earlier rounds
 
   const uint64_t q_desc0 = smem_desc(sQ, 16, 1024, kSwizzle128);
   const uint64_t q_tail0 = smem_desc(sQ + G::kQTail, 16, 256, kSwizzle32);
@@ -550,6 +554,7 @@ __device__ void mma_role(const AttnParams& p, uint32_t tmem, uint32_t sQ, uint32
         if (G::kHasTail) mma_ts(o_tmem + 64, p_tmem + kk * 8, vt + kk * 32, kIdescPVTail, acc);
       }
       mma_commit(bar.o_prog(s));
+      mbar_arrive(bar.pv_issued(s));
     }
     __syncwarp();
     VLA_TRACE_EVENT(kTrMmaPVDone, s, j);
@@ -566,9 +571,20 @@ __device__ void mma_role(const AttnParams& p, uint32_t tmem, uint32_t sQ, uint32
     RingPos cur = p.reuse ? unit_pos : pos;  // K/V event of the next (block, slot)
     if (score_warp) {
       // S of block j for slot s as soon as slot s has read S of block j-1.
+      // A round's first S waits until the slot's last P V of the previous
+      // round has been issued: the tensor pipe runs in issue order, and that
+      // P V gates the slot's epilogue, which comes before the new S is needed.
       for (int j = 0; ok && j < nb; ++j) {
         for (int s = 0; ok && s < ns; ++s) {
           if ((!sh || s == 0) && !(ok = wait_k(cur))) break;
+          if (j == 0) {
+            // No later P V of slot s can be issued before this S, so the
+            // barrier is at most one phase ahead of the one waited for.
+            const uint32_t npv = s == 0 ? npv0 : npv1;
+            if (npv > 0 && !(ok = wait_bounded(bar.pv_issued(s), (npv - 1u) & 1u, abort_flag,
+                                               lim, kSiteMmaPvIssued)))
+              break;
+          }
           if (!(ok = (j == 0 ? wait_q(s) : wait_free(s)))) break;
           scores(s, j, cur.slot);
           if (j == nb - 1) commit(bar.q_empty(s == 0 ? qi0 : qi1));
@@ -586,6 +602,8 @@ __device__ void mma_role(const AttnParams& p, uint32_t tmem, uint32_t sQ, uint32
       if (!ok) break;
       for (int s = 0; ok && s < ns; ++s) ok = wait_free(s);  // last block read out
       if (!ok) break;
+      npv0 += static_cast<uint32_t>(nb);
+      if (ns == 2) npv1 += static_cast<uint32_t>(nb);
     } else {
       // P V of block j for slot s as soon as slot s has stored P of block j.
       for (int j = 0; ok && j < nb; ++j) {
@@ -934,6 +952,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
     mbar_init(bar.drain(0), 1);
     mbar_init(bar.drain(1), 1);
     mbar_init(bar.never(), 1);
+    mbar_init(bar.pv_issued(0), 1);
+    mbar_init(bar.pv_issued(1), 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
