@@ -669,8 +669,14 @@ def run_block(args) -> None:
         rec["half_block_us"] = t_half
         rec["half_block_tflops"] = (fq + fo + c.flops()) / t_half / 1e6
         layer_flops = fq + fo + 2.0 * ff + c.flops()
-        t_layer = med(lambda: (ln(), lq(), at(), lo(), ln2(), f1(), f2()))
+        # Seconds of back-to-back GEMMs can run into the power cap: the layer's
+        # timing carries the SM clocks and throttle reasons seen while it ran.
+        with ClockSampler(torch.cuda.current_device()) as clocks:
+            clocks.mark_start()
+            t_layer = med(lambda: (ln(), lq(), at(), lo(), ln2(), f1(), f2()))
+            clocks.mark_end()
         rec["layer_us"] = t_layer
+        rec["layer_clocks"] = clocks.summary()
         rec["layer_tflops"] = layer_flops / t_layer / 1e6
         if not big:
             # The encoder's L whole layers (fresh weights and activations per layer) in one
