@@ -91,11 +91,13 @@ int vla_attn_fwd(const void* q, const void* k, const void* v, void* o,
  * packed [B, N, 3, H, d] bf16 input from `qkv_host` into the caller's device
  * buffer `qkv_dev`, runs vla_attn_fwd on it into `o_dev`, and copies the
  * [B, N, H, d] bf16 result back to `o_host`.  A batch of at least two chunks
- * (a chunk = the fewest whole images with 4 heads per SM) is pipelined per
- * chunk: input copy and kernel on `stream`, result copy on an internal
- * copy-out stream of the device, so that it overlaps the next chunk's input
- * copy; `stream` then waits for the copy-out stream.  Smaller batches use one
- * copy per direction on `stream`.  Either way the results are those of
+ * (a chunk = the fewest whole images with one head per SM) is pipelined per
+ * chunk: the input copies back to back on an internal copy-in stream of the
+ * device (after the earlier work of `stream`), each chunk's kernel on
+ * `stream` once its input has landed, its result copy on an internal
+ * copy-out stream, so that copies in both directions and the kernels
+ * overlap; `stream` then waits for both internal streams.  Smaller batches
+ * use one copy per direction on `stream`.  Either way the results are those of
  * vla_attn_fwd on the whole batch, and the host result is valid once
  * `stream` has been synchronised.  Host buffers should be pinned
  * (cudaHostAlloc / cudaHostRegister) for the copies to be asynchronous.
@@ -104,8 +106,8 @@ int vla_attn_fwd(const void* q, const void* k, const void* v, void* o,
  * inside one device allocation each, and they must not overlap) before the
  * first copy is enqueued, so an argument error leaves nothing enqueued.
  * Allocates no memory;
- * the first pipelined call on a device creates the copy-out stream and two
- * events, which live as long as the process.  Calls are serialised on a
+ * the first pipelined call on a device creates the two internal streams and
+ * five events, which live as long as the process.  Calls are serialised on a
  * library lock while they enqueue.
  */
 int vla_attn_fwd_host(const void* qkv_host, void* o_host, void* qkv_dev, void* o_dev,

@@ -239,14 +239,16 @@ def test_host_buffer_entry():
     assert_parity(got, want, "host-buffer entry")
 
 
-def test_host_buffer_entry_pipelined_chunks():
-    """A batch of several chunks takes the pipelined host path (copy-out stream): the
-    host result equals the device entry's bytes, on two calls in a row."""
+@pytest.mark.parametrize("full_chunks", [2, 7])
+def test_host_buffer_entry_pipelined_chunks(full_chunks):
+    """A batch of several chunks (a chunk = the fewest whole images with one head per SM)
+    takes the pipelined host path (copy-in and copy-out streams): the host result equals
+    the device entry's bytes on the whole batch, on two calls in a row."""
     import vit_self_attention_b200 as vab
     sm = torch.cuda.get_device_properties(0).multi_processor_count
     H, N, d = 16, 197, 64
-    chunk = -(-4 * sm // H)
-    B = 2 * chunk + 3  # two full chunks and a ragged one
+    chunk = -(-sm // H)
+    B = full_chunks * chunk + 3  # full chunks and a ragged one
     bits = si.packed_qkv(B, N, H, d, seed=4242)
     scale = 1.0 / math.sqrt(d)
     host_in = torch.from_numpy(bits.view(np.int16).copy()).pin_memory()

@@ -111,9 +111,13 @@ void set_dependent_launch(cudaLaunchConfig_t* cfg, cudaLaunchAttribute (&attr)[1
 // one set per device, created on first use (guarded by g_pipe_mutex, which
 // the caller holds for the whole enqueue sequence).
 struct HostPipe {
-  cudaStream_t out = nullptr;
-  cudaEvent_t fork = nullptr;
-  cudaEvent_t join = nullptr;
+  cudaStream_t in = nullptr;   // input copies, back to back
+  cudaStream_t out = nullptr;  // result copies
+  cudaEvent_t start = nullptr;    // `stream`'s earlier work -> copy-in stream
+  cudaEvent_t loaded = nullptr;   // a chunk's input copy -> its kernel on `stream`
+  cudaEvent_t fork = nullptr;     // a chunk's kernel -> its result copy
+  cudaEvent_t join = nullptr;     // copy-out stream -> `stream`
+  cudaEvent_t in_join = nullptr;  // copy-in stream -> `stream`
 };
 
 std::mutex g_pipe_mutex;
@@ -122,19 +126,20 @@ HostPipe g_pipe[kMaxDevices];
 int host_pipe(int dev, HostPipe** out) {
   HostPipe& p = g_pipe[dev];
   if (p.out == nullptr) {
-    cudaStream_t s = nullptr;
-    cudaEvent_t f = nullptr, j = nullptr;
-    if (cudaStreamCreateWithFlags(&s, cudaStreamNonBlocking) != cudaSuccess)
-      return VLA_ATTN_ERR_CUDA;
-    if (cudaEventCreateWithFlags(&f, cudaEventDisableTiming) != cudaSuccess ||
-        cudaEventCreateWithFlags(&j, cudaEventDisableTiming) != cudaSuccess) {
-      if (f != nullptr) cudaEventDestroy(f);
-      cudaStreamDestroy(s);
+    HostPipe n;
+    bool ok = cudaStreamCreateWithFlags(&n.in, cudaStreamNonBlocking) == cudaSuccess &&
+              cudaStreamCreateWithFlags(&n.out, cudaStreamNonBlocking) == cudaSuccess;
+    cudaEvent_t* evs[5] = {&n.start, &n.loaded, &n.fork, &n.join, &n.in_join};
+    for (cudaEvent_t* e : evs)
+      ok = ok && cudaEventCreateWithFlags(e, cudaEventDisableTiming) == cudaSuccess;
+    if (!ok) {
+      for (cudaEvent_t* e : evs)
+        if (*e != nullptr) cudaEventDestroy(*e);
+      if (n.in != nullptr) cudaStreamDestroy(n.in);
+      if (n.out != nullptr) cudaStreamDestroy(n.out);
       return VLA_ATTN_ERR_CUDA;
     }
-    p.out = s;
-    p.fork = f;
-    p.join = j;
+    p = n;
   }
   *out = &p;
   return VLA_ATTN_OK;
@@ -498,9 +503,12 @@ int vla_attn_fwd_host(const void* qkv_host, void* o_host, void* qkv_dev, void* o
       return rc;
     if (out_lo < in_hi && in_lo < out_hi) return VLA_ATTN_ERR_MEMORY;
   }
-  // Chunks of whole images, each with at least 4 heads per SM so that every
-  // launch still fills the GPU; a batch smaller than two chunks goes in one.
-  const long long min_heads = 4ll * di.sm_count;
+  // Chunks of whole images with at least one head per SM: a chunk's kernel
+  // is far shorter than the next chunk's input copy, so its efficiency does
+  // not matter, while a small last chunk keeps short the part of the step
+  // that nothing overlaps (its kernel and result copy).  A batch smaller than
+  // two chunks goes in one.
+  const long long min_heads = di.sm_count;
   const int chunk = static_cast<int>((min_heads + H - 1) / H);
   if (B < 2 * chunk) {
     if (cudaMemcpyAsync(qkv_dev, qkv_host, img_in * B, cudaMemcpyHostToDevice, st) != cudaSuccess)
@@ -511,10 +519,11 @@ int vla_attn_fwd_host(const void* qkv_host, void* o_host, void* qkv_dev, void* o
       return VLA_ATTN_ERR_CUDA;
     return VLA_ATTN_OK;
   }
-  // Pipelined: chunk i's host-to-device copy and kernel on `stream`, its
-  // device-to-host copy on the device's copy-out stream, so it overlaps the
-  // next chunk's host-to-device copy (the two directions use separate copy
-  // engines).  `stream` waits for the copy-out stream at the end.
+  // Pipelined: the input copies run back to back on the device's copy-in
+  // stream (after `stream`'s earlier work), chunk i's kernel on `stream` once
+  // its copy has landed, its result copy on the copy-out stream once the
+  // kernel is done; the two directions use separate copy engines.  `stream`
+  // waits for both side streams at the end.
   std::lock_guard<std::mutex> lock(g_pipe_mutex);
   HostPipe* pipe = nullptr;
   if ((rc = host_pipe(dev, &pipe)) != VLA_ATTN_OK) return rc;
@@ -523,11 +532,18 @@ int vla_attn_fwd_host(const void* qkv_host, void* o_host, void* qkv_dev, void* o
   char* din = static_cast<char*>(qkv_dev);
   char* dout = static_cast<char*>(o_dev);
   bool forked = false;
+  if (cudaEventRecord(pipe->start, st) != cudaSuccess ||
+      cudaStreamWaitEvent(pipe->in, pipe->start, 0) != cudaSuccess)
+    return VLA_ATTN_ERR_CUDA;
+  bool loading = false;
   for (int b0 = 0; b0 < B && rc == VLA_ATTN_OK; b0 += chunk) {
     const int nbi = B - b0 < chunk ? B - b0 : chunk;
     const size_t in_off = img_in * b0, out_off = img_out * b0;
-    if (cudaMemcpyAsync(din + in_off, hin + in_off, img_in * nbi, cudaMemcpyHostToDevice, st) !=
-        cudaSuccess) {
+    loading = true;
+    if (cudaMemcpyAsync(din + in_off, hin + in_off, img_in * nbi, cudaMemcpyHostToDevice,
+                        pipe->in) != cudaSuccess ||
+        cudaEventRecord(pipe->loaded, pipe->in) != cudaSuccess ||
+        cudaStreamWaitEvent(st, pipe->loaded, 0) != cudaSuccess) {
       rc = VLA_ATTN_ERR_CUDA;
       break;
     }
@@ -545,10 +561,13 @@ int vla_attn_fwd_host(const void* qkv_host, void* o_host, void* qkv_dev, void* o
                         pipe->out) != cudaSuccess)
       rc = VLA_ATTN_ERR_CUDA;
   }
-  // Join even after an error, so that work already on the copy-out stream is
+  // Join even after an error, so that work already on the side streams is
   // ordered before anything later on `stream`.
   if (forked && (cudaEventRecord(pipe->join, pipe->out) != cudaSuccess ||
                  cudaStreamWaitEvent(st, pipe->join, 0) != cudaSuccess))
+    rc = VLA_ATTN_ERR_CUDA;
+  if (loading && (cudaEventRecord(pipe->in_join, pipe->in) != cudaSuccess ||
+                  cudaStreamWaitEvent(st, pipe->in_join, 0) != cudaSuccess))
     rc = VLA_ATTN_ERR_CUDA;
   return rc;
 }
