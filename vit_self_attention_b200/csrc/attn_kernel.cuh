@@ -37,7 +37,9 @@
 // round, so instead a CTA walks the tiles of its heads two at a time across
 // head boundaries: the round that pairs the last tile of one head with the
 // first of the next streams both heads' K/V blocks through the ring (one load
-// per slot and block), the others one load per block shared by both slots.
+// per slot and block), the others one load per block shared by both slots;
+// when a head's blocks fit the ring, consecutive rounds of one head load them
+// once (`carry`).
 //
 // Pipelining.  A softmax thread signals "S consumed" as soon as it has the S
 // row of block j in registers, so the tensor core computes S of block j+1
@@ -160,7 +162,8 @@ struct AttnParams {
   int units_per_head;
   int num_units;
   int ring;                // K/V ring slots (<= kMaxRing)
-  int reuse;               // 1 when num_kblocks <= ring: a unit loads its K/V once
+  int reuse;               // 1 when num_kblocks <= ring (not stream mode): a unit loads
+                           // its K/V once
   float c;                 // scale * log2(e)
   unsigned long long wait_limit_ns;
   int test_stall;          // testing hook: softmax warps wait on a barrier nothing completes
@@ -168,6 +171,8 @@ struct AttnParams {
                            // (whole heads with an odd tile count), K/V streamed
   int qbuf;                // Q buffers per slot (1 or 2): with 2 the next round's Q tile
                            // loads while the current round runs
+  int carry;               // stream mode with a head's K/V blocks fitting the ring: rounds
+                           // of one head in a row load those blocks once
   __nv_bfloat16* o;        // [B, N, H, d] (the row stores of the kernel without staging)
 };
 
@@ -300,7 +305,12 @@ __device__ __forceinline__ Round next_round(const AttnParams& p, Cursor& c) {
     }
     x.t1 = tb;
     x.shared_kv = ub == c.u;
-    x.first = x.last = true;
+    // Consecutive rounds whose two tiles share a head (tiles 0-1, 2-3, ...)
+    // form a run: with `carry` the run loads its K/V blocks once and its later
+    // rounds read them from the ring; a round that pairs two heads, or a lone
+    // last tile, is a run of its own.
+    x.first = !(x.shared_kv && x.nslots == 2 && x.t0 >= 2);
+    x.last = !(x.shared_kv && x.nslots == 2 && x.t0 + 3 < p.num_qtiles);
     // Advance two tiles.
     c.u = ub;
     c.tq = tb + 1;
@@ -391,7 +401,8 @@ __device__ void load_role(const AttnParams& p, uint32_t sQ, uint32_t sK, uint32_
 
   for (Cursor cu = cursor_start(); ok && cursor_more(p, cu);) {
     const Round x = next_round(p, cu);
-    if (!p.reuse || x.first) {
+    const bool reuse = p.reuse || (p.carry && x.shared_kv);
+    if (!reuse || x.first) {
       const int E = x.shared_kv ? nb : 2 * nb;
       for (int e = 0; ok && e < E; ++e) {
         const int se = x.shared_kv ? 0 : (e & 1);
@@ -567,8 +578,9 @@ __device__ void mma_role(const AttnParams& p, uint32_t tmem, uint32_t sQ, uint32
     if (x.first) unit_pos = pos;
     const int ns = x.nslots;
     const bool sh = x.shared_kv;
-    const bool release = !p.reuse || x.last;
-    RingPos cur = p.reuse ? unit_pos : pos;  // K/V event of the next (block, slot)
+    const bool reuse = p.reuse || (p.carry && x.shared_kv);
+    const bool release = !reuse || x.last;
+    RingPos cur = reuse ? unit_pos : pos;  // K/V event of the next (block, slot)
     if (score_warp) {
       // S of block j for slot s as soon as slot s has read S of block j-1.
       // A round's first S waits until the slot's last P V of the previous

@@ -430,6 +430,7 @@ int launch(const void* q, void* o, int B, int N, int H, float scale, cudaStream_
   prm.qbuf = qbuf;
   prm.o = static_cast<__nv_bfloat16*>(o);
   prm.reuse = (nb <= ring && !prm.stream) ? 1 : 0;
+  prm.carry = (nb <= ring && prm.stream) ? 1 : 0;
   prm.c = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
   const unsigned long long lim = g_wait_limit_ns.load();
   prm.wait_limit_ns = lim == 0 ? kDefaultWaitLimitNs : lim;
