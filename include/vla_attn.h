@@ -128,8 +128,8 @@ const char* vla_attn_strerror(int status);
  * ran out (the output of that launch is then undefined).  `site`, if non-NULL,
  * receives the code of the first wait that ran out (0 if none): 1-3 the TMA
  * producer (Q slot, K block, V block), 11-16 the tensor-core issuers (Q, K,
- * V, P, S read out, previous round's P V issued), 21-22 the softmax warps (S, P V progress), 31 a drain
- * wait, 41 the testing stall.  This extends the plain status call
+ * V, P, S read out, previous round's P V issued), 21-22 the softmax warps
+ * (S, P V progress), 31 a drain wait, 41 the testing stall.  This extends the plain status call
  * vla_attn_last_device_status(stream) by the optional `site` out-parameter
  * (pass NULL for the plain form).  The status word is always kept; reading
  * it costs a stream synchronisation, so call it outside timed regions.

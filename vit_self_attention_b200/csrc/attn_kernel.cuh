@@ -65,7 +65,9 @@
 // (bounded) for its own tensor-core work, and the tensor memory is freed.
 // Every barrier has one consumer role that waits on each of its phases in
 // order, and no barrier can complete twice before its consumer has waited,
-// so a parity wait never confuses two phases.
+// so a parity wait never confuses two phases.  The one barrier whose waiter
+// skips phases, "P V issued" (waited on only before a round's first S), is
+// never more than one phase past the phase waited for (see mma_role).
 #pragma once
 
 #include <cuda_bf16.h>
